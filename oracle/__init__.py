@@ -1,0 +1,50 @@
+"""fp64 CPU oracle for Adaptive Block-Sparse Attention (ASA / ASA_G).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it.
+The CUDA library never imports, links or calls anything here, and nothing here
+imports the CUDA library: the two share no code, tables or helpers.  The only
+shared module is the seeded input generator in ``inputs/``, which holds none of
+the method's arithmetic.
+
+Everything is plain NumPy in float64 (bf16 inputs are read as exact float64
+values).  Each function cites the passage of "Video-BLADE: Block-Sparse Attention
+Meets Step Distillation for Efficient Video Generation" (arXiv 2508.10774,
+section "Adaptive Block-Sparse Attention") it restates.
+
+Parity status per function (how each is pinned is in tests/test_oracle_*.py):
+  gilbert_order      pinned: bijection, unit steps, brute force over all grids
+                     up to 8x8x8, 1-D identity, textbook Hilbert curve on 2^m
+                     squares (up to symmetry), locality vs raster.  The absolute
+                     order relative to other Gilbert implementations is
+                     "parity unpinned" (the pages do not define the curve).
+  permute/unpermute  pinned: round trip, explicit index definition.
+  estimate_pimp      pinned: k=b closed form vs the dense softmax map, row sums,
+                     in-block permutation invariance.
+  build_mask         pinned: brute-force minimality over all subsets (nb=8),
+                     tau->0 keeps the argmax, tau=1 keeps all, monotone in tau.
+  asa_forward        pinned: tau=1 equals dense attention (torch SDPA fp64);
+                     any mask equals SDPA with the token-expanded block mask.
+  asa_g_forward      pinned: SDPA fp64 over Concat(K, MeanPool_n K) with the
+                     additive ln(n) mask; n=1 closed form.
+  asa_backward       pinned: torch.autograd of masked SDPA fp64; central finite
+                     differences on a tiny case.
+"""
+from .gilbert import gilbert_order  # noqa: F401
+from .asa_ref import (  # noqa: F401
+    block_sizes,
+    sample_offsets,
+    sample_rows,
+    permute,
+    unpermute,
+    estimate_pimp,
+    build_mask,
+    mask_to_csr,
+    mask_to_csr_transposed,
+    marginal_rows,
+    global_tokens,
+    round_to_bf16,
+    asa_forward,
+    asa_backward,
+    attention_flops,
+)

@@ -1,0 +1,319 @@
+"""fp64 reference of the ASA hot path (test infrastructure; see oracle/__init__.py).
+
+Source: "Video-BLADE: Block-Sparse Attention Meets Step Distillation for Efficient
+Video Generation" (arXiv 2508.10774), section "Adaptive Block-Sparse Attention":
+  * "Preprocessing"            -> permute / unpermute (with gilbert.gilbert_order)
+  * "Step 1: Efficient block importance estimation" -> estimate_pimp
+  * "Step 2.1: Sparse mask construction"            -> build_mask
+  * "Step 2.2: Computation", variant 1 (standard ASA) and variant 2 (ASA_G, global
+    tokens with the fixed additive ln(n) mask)      -> asa_forward
+  * the mask also restricts attention "during both training and inference" (end
+    of Step 2.1)                                    -> asa_backward (fixed mask)
+  * "Implementation details": b = 128, k = 16.
+
+Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
+  * blocks are consecutive runs of b permuted tokens; the last block is ragged,
+    nothing is padded;
+  * the k "representative tokens" of a block of L tokens are the evenly strided
+    offsets floor(j L / k_I), j < k_I = min(k, L) (all tokens when L < k);
+  * P_approx is one softmax over all sampled keys of the head (the definition of
+    P = softmax(QK^T / sqrt(d)) is global); P_imp[I, J] is the max of the
+    k_I x k_J tile of P_approx;
+  * each row of P_imp is normalised to shares R = P_imp / sum(P_imp); the kept set
+    is the first c* blocks in (R descending, J ascending) order, c* the least c
+    whose cumulative share is >= tau; tau >= 1 keeps every block;
+  * ASA_G global token g is the mean of K (V) over permuted positions
+    [n g, min(n g + n, N)), rounded to bf16 (the kernels store bf16 operands);
+    every query sees every global token with logit q.kg / sqrt(d) + ln(n), also
+    for the ragged last window;
+  * LSE is the natural-log log-sum-exp of the logits a query row attends to.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------
+# blocking and sampling ("Preprocessing", "Step 1", "Implementation details")
+# ----------------------------------------------------------------------------
+
+def block_sizes(N: int, b: int = 128) -> list[int]:
+    """L_I for each block I: runs of b permuted tokens, the last one ragged."""
+    nb = -(-N // b)
+    return [min(b, N - b * I) for I in range(nb)]
+
+
+def sample_offsets(L: int, k: int = 16) -> list[int]:
+    """Offsets inside a block of L tokens of its k_I = min(k, L) sampled tokens."""
+    kk = min(k, L)
+    return [(j * L) // kk for j in range(kk)]
+
+
+def sample_rows(N: int, b: int = 128, k: int = 16) -> np.ndarray:
+    """Permuted positions of all sampled tokens, block by block (length M)."""
+    rows = []
+    for I, L in enumerate(block_sizes(N, b)):
+        rows.extend(b * I + s for s in sample_offsets(L, k))
+    return np.asarray(rows, dtype=np.int64)
+
+
+def _sample_block_starts(N: int, b: int, k: int) -> np.ndarray:
+    starts, pos = [], 0
+    for L in block_sizes(N, b):
+        starts.append(pos)
+        pos += min(k, L)
+    return np.asarray(starts, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# token rearrangement ("Preprocessing")
+# ----------------------------------------------------------------------------
+
+def permute(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x [B, N, H, d] in raster order -> xp [B, H, N, d] with xp[b,h,i] = x[b,perm[i],h]."""
+    return np.ascontiguousarray(np.transpose(x[:, perm, :, :], (0, 2, 1, 3)))
+
+
+def unpermute(xp: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Inverse of permute: x[b, perm[i], h] = xp[b, h, i]."""
+    B, H, N, d = xp.shape
+    x = np.empty((B, N, H, d), dtype=xp.dtype)
+    x[:, perm, :, :] = np.transpose(xp, (0, 2, 1, 3))
+    return x
+
+
+# ----------------------------------------------------------------------------
+# Step 1: block importance estimation
+# ----------------------------------------------------------------------------
+
+def estimate_pimp(qp: np.ndarray, kp: np.ndarray, b: int = 128, k: int = 16) -> np.ndarray:
+    """P_imp [B, H, nb, nb] from k sampled tokens per block.
+
+    Q_s, K_s = sampled rows; P_approx = softmax(Q_s K_s^T / sqrt(d)) over each row;
+    P_imp[I, J] = max of the (rows of block I) x (columns of block J) tile.
+    With k >= b every token is sampled and this is the exact max-pool of the full
+    attention map that the section describes first.
+    """
+    B, H, N, d = qp.shape
+    rows = sample_rows(N, b, k)
+    starts = _sample_block_starts(N, b, k)
+    nb = len(starts)
+    out = np.empty((B, H, nb, nb), dtype=np.float64)
+    for bb in range(B):
+        for h in range(H):
+            Qs = np.asarray(qp[bb, h, rows, :], dtype=np.float64)
+            Ks = np.asarray(kp[bb, h, rows, :], dtype=np.float64)
+            S = (Qs @ Ks.T) / math.sqrt(d)
+            S = S - S.max(axis=1, keepdims=True)
+            P = np.exp(S)
+            P = P / P.sum(axis=1, keepdims=True)
+            tile_max = np.maximum.reduceat(np.maximum.reduceat(P, starts, axis=0), starts, axis=1)
+            out[bb, h] = tile_max
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Step 2.1: threshold mask
+# ----------------------------------------------------------------------------
+
+def _row_order(p_row: np.ndarray):
+    share = p_row / p_row.sum()
+    order = np.lexsort((np.arange(len(p_row)), -share))   # share desc, J asc
+    return share, order
+
+
+def _row_cut(share: np.ndarray, order: np.ndarray, tau: float) -> int:
+    nb = len(share)
+    if tau >= 1.0:
+        return nb
+    cum = np.cumsum(share[order])
+    hit = np.nonzero(cum >= tau)[0]
+    return int(hit[0]) + 1 if len(hit) else nb
+
+
+def build_mask(pimp: np.ndarray, tau: float) -> np.ndarray:
+    """Boolean block mask [B, H, nb, nb]: per row the fewest blocks with share >= tau."""
+    B, H, nb, _ = pimp.shape
+    mask = np.zeros(pimp.shape, dtype=bool)
+    for bb in range(B):
+        for h in range(H):
+            for I in range(nb):
+                share, order = _row_order(pimp[bb, h, I])
+                c = _row_cut(share, order, tau)
+                mask[bb, h, I, order[:c]] = True
+    return mask
+
+
+def marginal_rows(pimp: np.ndarray, tau: float, eps: float = 1e-4,
+                  tie_eps: float = 1e-6) -> np.ndarray:
+    """Rows whose cut an fp32 evaluation may legitimately place differently.
+
+    A row is marginal when the cumulative share at the cut, or one block before
+    it, lies within ``eps`` of tau, or when the last kept share and the first
+    dropped share differ by less than ``tie_eps``.
+    """
+    B, H, nb, _ = pimp.shape
+    marg = np.zeros((B, H, nb), dtype=bool)
+    if tau >= 1.0:
+        return marg
+    for bb in range(B):
+        for h in range(H):
+            for I in range(nb):
+                share, order = _row_order(pimp[bb, h, I])
+                cum = np.cumsum(share[order])
+                c = _row_cut(share, order, tau)
+                ncol = len(share)
+                m = abs(cum[c - 1] - tau) < eps
+                if c >= 2:
+                    m |= abs(cum[c - 2] - tau) < eps
+                if c < ncol:
+                    m |= abs(share[order[c - 1]] - share[order[c]]) < tie_eps
+                marg[bb, h, I] = m
+    return marg
+
+
+def mask_to_csr(mask: np.ndarray):
+    """row_ptr [B*H*nb + 1], col_idx [nnz]; rows in (b, h, I) order, columns ascending."""
+    B, H, nb, _ = mask.shape
+    flat = mask.reshape(B * H * nb, nb)
+    counts = flat.sum(axis=1)
+    row_ptr = np.zeros(B * H * nb + 1, dtype=np.int64)
+    row_ptr[1:] = np.cumsum(counts)
+    col_idx = np.nonzero(flat)[1].astype(np.int64)
+    return row_ptr, col_idx
+
+
+def mask_to_csr_transposed(mask: np.ndarray):
+    """col_ptr [B*H*nb + 1], row_idx [nnz]: for each (b, h, J) the q-blocks I keeping J."""
+    return mask_to_csr(np.swapaxes(mask, 2, 3))
+
+
+# ----------------------------------------------------------------------------
+# Step 2.2: computation (standard ASA and ASA_G), and its backward
+# ----------------------------------------------------------------------------
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value (ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                  # x = m * 2**e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)   # 8 significant bits
+
+
+def global_tokens(x_head: np.ndarray, n: int) -> np.ndarray:
+    """MeanPool_n over permuted positions of one head's [N, d] rows, bf16-rounded."""
+    N = x_head.shape[0]
+    G = -(-N // n)
+    out = np.empty((G, x_head.shape[1]), dtype=np.float64)
+    for g in range(G):
+        out[g] = np.asarray(x_head[n * g:min(n * g + n, N)], dtype=np.float64).mean(axis=0)
+    return round_to_bf16(out)
+
+
+def _kept_positions(mask_row: np.ndarray, N: int, b: int) -> np.ndarray:
+    blocks = np.nonzero(mask_row)[0]
+    if len(blocks) == 0:
+        return np.zeros(0, dtype=np.int64)
+    return np.concatenate([np.arange(b * J, min(b * J + b, N)) for J in blocks])
+
+
+def asa_forward(qp, kp, vp, mask, b: int = 128, global_window: int = 0,
+                q_index: Iterable[int] | None = None):
+    """O [B, H, nq, d] and natural-log LSE [B, H, nq] for the queries ``q_index``.
+
+    A query in block I attends to every token of the kept blocks of row I (standard
+    ASA).  With ``global_window = n > 0`` (ASA_G) it also attends to all
+    ceil(N/n) global tokens, whose logits carry the fixed additive ln(n).
+    """
+    B, H, N, d = qp.shape
+    q_index = np.arange(N) if q_index is None else np.asarray(list(q_index), dtype=np.int64)
+    nq = len(q_index)
+    O = np.zeros((B, H, nq, d), dtype=np.float64)
+    LSE = np.zeros((B, H, nq), dtype=np.float64)
+    scale = 1.0 / math.sqrt(d)
+    qblk = q_index // b
+    for bb in range(B):
+        for h in range(H):
+            if global_window > 0:
+                Kg = global_tokens(kp[bb, h], global_window)
+                Vg = global_tokens(vp[bb, h], global_window)
+            for I in np.unique(qblk):
+                sel = np.nonzero(qblk == I)[0]
+                q = np.asarray(qp[bb, h, q_index[sel]], dtype=np.float64)
+                idx = _kept_positions(mask[bb, h, I], N, b)
+                K = np.asarray(kp[bb, h, idx], dtype=np.float64)
+                V = np.asarray(vp[bb, h, idx], dtype=np.float64)
+                S = (q @ K.T) * scale
+                if global_window > 0:
+                    S = np.concatenate([S, (q @ Kg.T) * scale + math.log(global_window)], axis=1)
+                    V = np.concatenate([V, Vg], axis=0)
+                m = S.max(axis=1, keepdims=True)
+                E = np.exp(S - m)
+                l = E.sum(axis=1, keepdims=True)
+                O[bb, h, sel] = (E / l) @ V
+                LSE[bb, h, sel] = (m + np.log(l))[:, 0]
+    return O, LSE
+
+
+def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
+                 q_blocks=None, kv_blocks=None):
+    """Gradients of standard ASA under a fixed mask (the mask is not differentiated).
+
+    For each query block I with kept keys K_I, V_I:
+        P = softmax(Q_I K_I^T / sqrt(d)),  dV_I += P^T dO_I,  dP = dO_I V_I^T,
+        dS = P * (dP - rowsum(P * dP)),    dQ_I = dS K_I / sqrt(d),
+        dK_I += dS^T Q_I / sqrt(d).
+    Returns dicts {(b, h, I): dQ block} and {(b, h, J): (dK block, dV block)} for
+    the requested heads / blocks (all by default).
+    """
+    B, H, N, d = qp.shape
+    nb = -(-N // b)
+    scale = 1.0 / math.sqrt(d)
+    heads = [(bb, h) for bb in range(B) for h in range(H)] if heads is None else list(heads)
+    dq_out, dkv_out = {}, {}
+    for (bb, h) in heads:
+        want_q = set(range(nb)) if q_blocks is None else set(q_blocks)
+        want_kv = set(range(nb)) if kv_blocks is None else set(kv_blocks)
+        dK = {J: np.zeros((min(b, N - b * J), d)) for J in want_kv}
+        dV = {J: np.zeros((min(b, N - b * J), d)) for J in want_kv}
+        for I in range(nb):
+            kept = np.nonzero(mask[bb, h, I])[0]
+            if I not in want_q and not (set(kept.tolist()) & want_kv):
+                continue
+            rows = np.arange(b * I, min(b * I + b, N))
+            idx = _kept_positions(mask[bb, h, I], N, b)
+            Q = np.asarray(qp[bb, h, rows], dtype=np.float64)
+            K = np.asarray(kp[bb, h, idx], dtype=np.float64)
+            V = np.asarray(vp[bb, h, idx], dtype=np.float64)
+            dO = np.asarray(dout[bb, h, rows], dtype=np.float64)
+            S = (Q @ K.T) * scale
+            E = np.exp(S - S.max(axis=1, keepdims=True))
+            P = E / E.sum(axis=1, keepdims=True)
+            dP = dO @ V.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            if I in want_q:
+                dq_out[(bb, h, I)] = (dS @ K) * scale
+            off = 0
+            for J in kept:
+                LJ = min(b, N - b * J)
+                if J in want_kv:
+                    dK[J] += (dS[:, off:off + LJ].T @ Q) * scale
+                    dV[J] += P[:, off:off + LJ].T @ dO
+                off += LJ
+        for J in want_kv:
+            dkv_out[(bb, h, J)] = (dK[J], dV[J])
+    return dq_out, dkv_out
+
+
+def attention_flops(mask: np.ndarray, N: int, d: int, b: int = 128,
+                    global_window: int = 0) -> int:
+    """Effective forward FLOPs: 4 d L_I L_J per kept tile (+ 4 d N G per head for ASA_G)."""
+    L = np.asarray(block_sizes(N, b), dtype=np.int64)
+    tiles = (mask * (L[:, None] * L[None, :])).sum()
+    flops = 4 * d * int(tiles)
+    if global_window > 0:
+        B, H = mask.shape[:2]
+        flops += 4 * d * N * (-(-N // global_window)) * B * H
+    return flops
