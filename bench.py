@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""ASA benchmark: one attention call of the Wan2.1-1.3B-shaped workload per step.
+
+A step is the whole hot path of one training-free ASA self-attention call on
+resident inputs: Gilbert permute of Q, K, V -> sampled block-importance estimate ->
+tau-threshold mask (CSR) -> block-sparse attention forward -> unpermute of O.
+Prints ONE JSON line (rank 0).  Metric: effective TFLOP/s counting only kept tiles
+(4 d sum_kept L_I L_J per head), whole-job (all ranks) over the max-over-ranks time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own seeded batch on its own GPU (heads and
+batches are independent, no collective on the data path: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "wan2.1-1.3b"
+METRIC = "ASA ms/call & effective TFLOP/s at 32760 tok, H=12, d=128, τ=0.95"
+KERNELS_PER_STEP = 8   # permute3, est_logits, est_pool, mask_rows, scan, fill, fwd, unpermute
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d["bf16_tflops_sustained"], d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _kept_tile_flops(row_ptr, col_idx, B, H, N, d):
+    """4 d sum over kept (I, J) of L_I L_J, from the CSR the step produced."""
+    nb = -(-N // 128)
+    L = np.array([min(128, N - 128 * i) for i in range(nb)], dtype=np.int64)
+    rp = row_ptr.astype(np.int64)
+    counts = np.diff(rp)
+    rows_I = np.tile(np.arange(nb), B * H)
+    LJ = L[col_idx[:rp[-1]].astype(np.int64)]
+    per_row = np.add.reduceat(LJ, rp[:-1]) if rp[-1] > 0 else np.zeros(len(counts), np.int64)
+    per_row = np.where(counts > 0, per_row, 0)
+    return int(4 * d * (L[rows_I] * per_row).sum()), int(rp[-1]), B * H * nb * nb
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                clk, mx, pw = float(f[1]), float(f[2]), float(f[3])
+            except ValueError:
+                continue
+            n += 1
+            smax = mx
+            if pw > 250.0:   # under load
+                sm.append(clk)
+                for name, val in zip(names, f[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": n, "samples_under_load": len(sm)}
+
+
+def cpu_oracle_sample(wl, x, budget_s=15.0):
+    """Time the fp64 oracle on a bounded sample of the workload: estimate + mask of one
+    head, then the sparse forward of as many of its query blocks as fit the budget."""
+    import oracle
+    import threadpoolctl
+    perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
+    h = 0
+    t0 = time.perf_counter()
+    qp = oracle.permute(x["q"][:, :, h:h + 1].double().numpy(), perm)
+    kp = oracle.permute(x["k"][:, :, h:h + 1].double().numpy(), perm)
+    vp = oracle.permute(x["v"][:, :, h:h + 1].double().numpy(), perm)
+    pimp = oracle.estimate_pimp(qp, kp)
+    mask = oracle.build_mask(pimp, wl.tau)
+    t_mask = time.perf_counter() - t0
+    nb = mask.shape[-1]
+    flops, blocks, t_fwd = 0, 0, 0.0
+    L = oracle.block_sizes(wl.N)
+    order = np.random.default_rng(0).permutation(nb)
+    for I in order:
+        t1 = time.perf_counter()
+        oracle.asa_forward(qp, kp, vp, mask, q_index=np.arange(128 * I, 128 * I + L[I]))
+        t_fwd += time.perf_counter() - t1
+        flops += 4 * wl.d * L[I] * sum(L[J] for J in np.nonzero(mask[0, 0, I])[0])
+        blocks += 1
+        if t_mask + t_fwd > budget_s:
+            break
+    # the sample's per-head share of estimate+mask is charged in proportion
+    t_total = t_fwd + t_mask * blocks / nb
+    info = threadpoolctl.threadpool_info()
+    cores = max([i.get("num_threads", 1) for i in info] or [1])
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": (f"1 of {wl.H} heads: fp64 estimate+mask of the head ({t_mask:.1f} s, charged "
+                       f"{blocks}/{nb} of it) + sparse forward of {blocks} of {nb} query blocks "
+                       f"({t_fwd:.1f} s)")}
+
+
+def run_reference(args, wl):
+    """The reference arm: the fp64 CPU oracle, timed as it stands, on a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from inputs import make_inputs
+    x = make_inputs(wl)
+    vals = []
+    for step in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(wl, x, budget_s=args.ref_budget)
+        if step >= args.warmup:
+            vals.append(r)
+    v = statistics.median(r["value"] for r in vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl),
+        "cpu_baseline": {**vals[-1], "value": v},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def _config(wl):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "d": wl.d, "N": wl.N,
+            "grid_THW": [wl.T, wl.Hg, wl.W], "block": 128, "samples": 16, "tau": wl.tau,
+            "l2": "inputs larger than L2: raster Q, K, V are 3 x 100.6 MB",
+            "parallelism": "one independent call per GPU (weak)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from inputs import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from video_dit_dynamic_gilbert_b200 import asa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    x = make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    B, N, H, d = q.shape
+    T, Hg, W = wl.T, wl.Hg, wl.W
+    qp, kp, vp = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    op = torch.empty_like(qp)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    ws = asa.estimate_mask_workspace(B, H, N, dev)
+    mask = asa._alloc_mask(B, H, N, dev, transposed=False)
+    stream = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        asa.asa_gilbert_permute3(q, k, v, T, Hg, W, outs=(qp, kp, vp))
+        if marks is not None:
+            marks[1].record(stream)
+        asa.asa_estimate_mask(qp, kp, wl.tau, transposed=False, workspace=ws, mask=mask)
+        if marks is not None:
+            marks[2].record(stream)
+        asa.asa_sparse_attn_fwd(qp, kp, vp, mask, out=op, lse=lse)
+        if marks is not None:
+            marks[3].record(stream)
+        asa.asa_unpermute(op, T, Hg, W, out=out)
+        if marks is not None:
+            marks[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flops, nnz, tiles = _kept_tile_flops(mask.row_ptr.cpu().numpy(), mask.col_idx.cpu().numpy(),
+                                         B, H, N, d)
+
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    start, stop = ev(), ev()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(marks[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        f = torch.tensor([float(flops)], device=dev, dtype=torch.float64)
+        dist.all_reduce(f)
+        total_flops = float(f.item())
+    else:
+        total_flops = float(flops)
+
+    ms_step = elapsed_ms / args.steps
+    stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
+    st_ms = stage.mean(axis=0)
+    fwd_ms = float(st_ms[2])
+    value = total_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    burst, sustained, hbm, peak_kind = _peaks()
+    achieved = flops / (fwd_ms * 1e-3) / 1e12
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": _config(wl),
+        "stages_ms": {"permute_qkv": float(st_ms[0]), "estimate_mask": float(st_ms[1]),
+                      "attn_fwd": fwd_ms, "unpermute": float(st_ms[3])},
+        "kept_tiles": nnz, "tiles": tiles, "kept_fraction": nnz / tiles,
+        "effective_flops_per_call": flops,
+        "roofline": {"kernel": "asa sparse attention forward", "bound": "tensor",
+                     "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst, "traffic": None,
+                     "peak_kind": f"{peak_kind} bf16 burst",
+                     "frac_of_sustained": achieved / sustained},
+        "clocks": clk,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+    }
+
+    # ---- end to end through the public call, host buffers in and out
+    qh, kh, vh = (x[n].pin_memory() for n in ("q", "k", "v"))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    e_times = []
+    for i in range(args.e2e_steps + 2):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+        o_d, _, _ = asa.asa_attention(qd, kd, vd, T, Hg, W, wl.tau)
+        oh.copy_(o_d, non_blocking=True)
+        torch.cuda.synchronize()
+        if i >= 2:
+            e_times.append(time.perf_counter() - t0)
+    e_s = statistics.median(e_times)
+    if world > 1:
+        t = torch.tensor([e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_s = float(t.item())
+    nbytes = q.numel() * q.element_size()
+    result["e2e"] = {"value": total_flops / e_s / 1e12, "unit": "TFLOP/s",
+                     "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+                     "ms_per_call": e_s * 1e3}
+
+    if not args.no_extras:
+        result["extras"] = extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_oracle_sample(wl, x)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
+    """Context measured after the timed region: dense attention on the same GPU (our
+    kernel with every tile kept, and torch SDPA), ASA_G and the backward."""
+    import torch
+    B, H, N, d = qp.shape
+
+    def timeit(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    dense_flops = 4 * d * N * N * B * H
+    p = torch.ones((B, H, -(-N // 128), -(-N // 128)), dtype=torch.float32, device=dev)
+    full = asa.asa_build_mask(p, N, 1.0, transposed=True)
+    ours_dense = timeit(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, full))
+    sdpa = timeit(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp))
+    tmask = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
+    g_ms = timeit(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, tmask, global_window=64))
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, tmask)
+    dout = torch.randn_like(qp)
+    bwd_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, tmask), reps=5)
+    flops, _, _ = _kept_tile_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
+                                   B, H, N, d)
+    G = -(-N // 64)
+    return {
+        "dense_ours_fwd_ms": ours_dense, "dense_ours_tflops": dense_flops / ours_dense / 1e9,
+        "dense_torch_sdpa_ms": sdpa, "dense_torch_sdpa_tflops": dense_flops / sdpa / 1e9,
+        "asa_g_fwd_ms_n64": g_ms,
+        "asa_g_fwd_tflops": (flops + 4 * d * N * G * B * H) / g_ms / 1e9,
+        "bwd_ms": bwd_ms, "bwd_tflops": 2.5 * flops / bwd_ms / 1e9,
+    }
+
+
+if __name__ == "__main__":
+    main()

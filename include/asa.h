@@ -1,0 +1,189 @@
+/*
+ * asa.h -- C ABI of the B200 (sm_100a) Adaptive Block-Sparse Attention library
+ * (libasa.so).
+ *
+ * The method is ASA from "Video-BLADE: Block-Sparse Attention Meets Step
+ * Distillation for Efficient Video Generation" (arXiv 2508.10774), section
+ * "Adaptive Block-Sparse Attention":
+ *   Preprocessing  -- Gilbert rearrangement of the (T, H, W) token grid, then
+ *                     blocks of b = 128 consecutive permuted tokens;
+ *   Step 1         -- block importance P_imp from k = 16 sampled tokens per block;
+ *   Step 2.1       -- per query block, the fewest key blocks whose cumulative share
+ *                     of P_imp reaches tau;
+ *   Step 2.2       -- attention over the kept (query block, key block) tiles only:
+ *                     standard ASA, or ASA_G with mean-pooled global tokens whose
+ *                     logits carry a fixed additive ln(n);
+ *   the same mask restricts the backward pass (end of Step 2.1).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are bf16 unless stated; "device" pointers are CUDA device memory
+ *     owned by the caller, "host" pointers are host memory owned by the caller.
+ *     The library never frees caller memory.
+ *   - Layouts: the model layout is raster [B, N, H, d] (token n = (t*Hg + y)*W + x);
+ *     the permuted layout is [B, H, N, d] (head-major, tokens in Gilbert order).
+ *     Rows are dense; every pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream; none synchronises the host except
+ *     the first call for a new (T, Hg, W) shape, which builds and uploads the
+ *     permutation table once (the library owns that table until asa_shutdown).
+ *   - Supported: head dim d in {64, 128}, block b = 128, samples k = 16,
+ *     N = number of tokens in [1, ASA_MAX_TOKENS].
+ *   - Return 0 (ASA_OK) or a negative ASA_ERR_* code; asa_last_error_string()
+ *     then describes the failure of the calling thread's last failing call.
+ *     Argument checks run on the host before anything is launched, so a
+ *     rejected call touches no device memory.
+ */
+#ifndef ASA_H_
+#define ASA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ASA_OK 0
+#define ASA_ERR_INVALID_ARG (-1) /* null/misaligned pointer, bad shape, N != T*Hg*W, tau <= 0 */
+#define ASA_ERR_UNSUPPORTED (-2) /* d not in {64,128}, block != 128, samples != 16, too large */
+#define ASA_ERR_WORKSPACE (-3)   /* workspace missing or smaller than the *_workspace_size() */
+#define ASA_ERR_CUDA (-4)        /* a CUDA call or kernel launch failed */
+#define ASA_ERR_TIMEOUT (-5)     /* a device-side bounded wait expired (see asa_check_device_status) */
+
+#define ASA_MAX_TOKENS 262144   /* N limit: at most 2048 blocks of 128 */
+#define ASA_BLOCK 128
+#define ASA_SAMPLES 16
+
+/* Library version as 10000*major + 100*minor + patch. */
+int asa_version(void);
+
+/* Message of the calling thread's last failing call ("" if none). Never NULL. */
+const char* asa_last_error_string(void);
+
+/*
+ * Gilbert order (Preprocessing paragraph): perm_host[i] = raster index of the token
+ * at curve position i, for the T x Hg x W grid.  perm_host: host, N = T*Hg*W int32.
+ * Pure host computation.  The curve is a generalised Hilbert curve whose
+ * consecutive cells are grid neighbours and which reduces to the Hilbert curve on
+ * 2^m x 2^m frames.
+ */
+int asa_gilbert_index(int T, int Hg, int W, int32_t* perm_host);
+
+/*
+ * Gather to Gilbert order (Preprocessing paragraph):
+ *   xp[b, h, i, :] = x[b, perm[i], h, :]
+ * x: device bf16 [B, N, H, d] raster; xp: device bf16 [B, H, N, d]; N = T*Hg*W.
+ * x and xp must not overlap.
+ */
+int asa_gilbert_permute(const void* x, void* xp, int B, int T, int Hg, int W, int H, int d,
+                        void* stream);
+
+/* Same gather applied to three tensors in one launch (Q, K and V of one call). */
+int asa_gilbert_permute3(const void* x0, const void* x1, const void* x2, void* xp0, void* xp1,
+                         void* xp2, int B, int T, int Hg, int W, int H, int d, void* stream);
+
+/*
+ * Inverse scatter back to raster order: x[b, perm[i], h, :] = xp[b, h, i, :].
+ * xp: device bf16 [B, H, N, d]; x: device bf16 [B, N, H, d].
+ */
+int asa_unpermute(const void* xp, void* x, int B, int T, int Hg, int W, int H, int d, void* stream);
+
+/*
+ * Workspace bytes needed by asa_estimate / asa_build_mask / asa_estimate_mask for
+ * this shape (device memory, any content on entry, 256-byte aligned).
+ */
+size_t asa_estimate_mask_workspace_size(int B, int H, int N);
+
+/*
+ * Step 1, block importance (P_imp) only.
+ * Block I holds permuted positions [128 I, min(128 I + 128, N)) of L_I tokens; its
+ * k_I = min(16, L_I) samples are offsets floor(j L_I / k_I).  With Q_s, K_s the
+ * sampled rows of qp, kp (M rows in block order),
+ *   P_approx = rowsoftmax(Q_s K_s^T / sqrt(d)),
+ *   P_imp[b, h, I, J] = max over the k_I x k_J tile (I, J) of P_approx.
+ * qp, kp: device bf16 [B, H, N, d]; p_imp: device fp32 [B, H, nb, nb], nb = ceil(N/128).
+ */
+int asa_estimate(const void* qp, const void* kp, int B, int H, int N, int d, int block,
+                 int samples, void* workspace, size_t ws_bytes, float* p_imp, void* stream);
+
+/*
+ * Step 2.1 from a given P_imp: per row (b, h, I), with shares R = P_imp / rowsum,
+ * keep the fewest key blocks whose cumulative share (shares in descending order,
+ * ties by lower J) reaches tau (tau >= 1 keeps all).  Emits the kept blocks as CSR:
+ *   row_ptr  device int32 [B*H*nb + 1], rows in (b, h, I) order;
+ *   col_idx  device int32, capacity B*H*nb*nb (upper bound), J ascending per row;
+ *   nnz_out  device int32 [1] = row_ptr[B*H*nb];
+ *   col_ptr_t, row_idx_t (both NULL or both set): the transposed CSR, for each
+ *            (b, h, J) the q-blocks I keeping J, ascending (same capacities);
+ *            the backward pass walks it.
+ * p_imp: device fp32 [B, H, nb, nb].  tau must be > 0.
+ */
+int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* workspace,
+                   size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                   int32_t* col_ptr_t, int32_t* row_idx_t, void* stream);
+
+/* Steps 1 + 2.1 in one call (P_imp stays in the workspace). Arguments as above. */
+int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d, int block,
+                      int samples, float tau, void* workspace, size_t ws_bytes, int32_t* row_ptr,
+                      int32_t* col_idx, int32_t* nnz_out, int32_t* col_ptr_t, int32_t* row_idx_t,
+                      void* stream);
+
+/*
+ * ASA_G global tokens (Step 2.2, variant 2): xg[b, h, g, :] = bf16(mean of
+ * xp[b, h, i, :] over permuted positions i in [n g, min(n g + n, N))), g < ceil(N/n).
+ * xp: device bf16 [B, H, N, d]; xg: device bf16 [B, H, ceil(N/n), d]; n >= 1.
+ */
+int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n, void* stream);
+
+/* Workspace bytes of asa_sparse_attn_fwd (0 for standard ASA). */
+size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window);
+
+/*
+ * Step 2.2, forward over the kept tiles only.  For a query i of block I:
+ *   O_i = softmax_j(q_i . k_j / sqrt(d)) V over the tokens j of the kept blocks
+ *   of row (b, h, I)  [standard ASA, global_window = 0];
+ * with global_window = n > 0 (ASA_G) the softmax also spans all ceil(N/n) global
+ * tokens (asa_global_pool of K and V, built in the workspace) with logits
+ * q_i . kg / sqrt(d) + ln(n).
+ * qp, kp, vp: device bf16 [B, H, N, d]; row_ptr/col_idx: the CSR of asa_build_mask;
+ * o: device bf16 [B, H, N, d]; lse: device fp32 [B, H, N], natural-log
+ * log-sum-exp of each row's logits (kept for the backward).
+ */
+int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                        const int32_t* col_idx, int B, int H, int N, int d, int block,
+                        int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
+                        void* stream);
+
+/* Workspace bytes of asa_sparse_attn_bwd. */
+size_t asa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward of standard ASA under the fixed mask (the mask is not differentiated):
+ *   P = exp(S - LSE), D = rowsum(dO * O), dV = P^T dO, dS = P * (dO V^T - D),
+ *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), all over kept tiles only.
+ * qp, kp, vp, o, dout: device bf16 [B, H, N, d]; lse: device fp32 [B, H, N] from the
+ * forward; row_ptr/col_idx and col_ptr_t/row_idx_t: both CSRs of asa_build_mask;
+ * dq, dk, dv: device bf16 [B, H, N, d] (fully written; no accumulation into them).
+ */
+int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
+                        const void* dout, const float* lse, const int32_t* row_ptr,
+                        const int32_t* col_idx, const int32_t* col_ptr_t,
+                        const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                        void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
+                        void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error word of
+ * the current device.  Returns ASA_OK, ASA_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last check, or ASA_ERR_CUDA on a CUDA error.
+ */
+int asa_check_device_status(void* stream);
+
+/* Frees the cached permutation tables of every device.  Safe to call twice. */
+void asa_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ASA_H_ */

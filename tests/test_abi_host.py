@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/asa.h declares, computes the Gilbert table exactly like the oracle,
+and rejects bad arguments with the documented codes before touching a device.
+
+Every call below is built to fail validation (or is pure host code), so nothing is
+ever launched with the fake pointers these tests pass."""
+import ctypes
+import itertools
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from video_dit_dynamic_gilbert_b200 import asa
+from video_dit_dynamic_gilbert_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "asa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return asa.lib()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(asa_\w+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(asa._SIGNATURES), set(names) ^ set(asa._SIGNATURES)
+
+
+def test_version_and_error_string(L):
+    assert L.asa_version() >= 100
+    assert isinstance(L.asa_last_error_string(), bytes)
+
+
+@pytest.mark.parametrize("shape", list(itertools.product([1, 2, 3, 5, 8], repeat=3)))
+def test_gilbert_table_matches_oracle_small(L, shape):
+    np.testing.assert_array_equal(asa.asa_gilbert_index(*shape), oracle.gilbert_order(*shape))
+
+
+@pytest.mark.parametrize("shape", [(21, 30, 52), (13, 30, 45), (21, 45, 80), (4, 16, 16),
+                                   (1, 64, 64), (7, 9, 11), (1, 2, 197)])
+def test_gilbert_table_matches_oracle_workloads(L, shape):
+    np.testing.assert_array_equal(asa.asa_gilbert_index(*shape), oracle.gilbert_order(*shape))
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+MIS = ctypes.c_void_p(0x10008)       # misaligned
+
+
+def test_gilbert_index_rejects(L):
+    buf = np.empty(8, dtype=np.int32)
+    p = buf.ctypes.data_as(ctypes.c_void_p)
+    assert L.asa_gilbert_index(0, 2, 2, p) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_gilbert_index(2, 2, 2, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_gilbert_index(1, 1, 300000, p) == asa.ASA_ERR_UNSUPPORTED
+    assert b"300000" in L.asa_last_error_string()
+
+
+def test_permute_rejects(L):
+    # bad head dim, aliasing, null, misaligned: all fail before any device work
+    assert L.asa_gilbert_permute(FAKE, ctypes.c_void_p(0x20000), 1, 2, 2, 2, 3, 96, None) == \
+        asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_gilbert_permute(FAKE, FAKE, 1, 2, 2, 2, 3, 64, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_gilbert_permute(None, FAKE, 1, 2, 2, 2, 3, 64, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_unpermute(MIS, FAKE, 1, 2, 2, 2, 3, 64, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_gilbert_permute(FAKE, ctypes.c_void_p(0x20000), 0, 2, 2, 2, 3, 64, None) == \
+        asa.ASA_ERR_INVALID_ARG
+    assert L.asa_gilbert_permute(FAKE, ctypes.c_void_p(0x20000), 1, 0, 2, 2, 3, 64, None) == \
+        asa.ASA_ERR_INVALID_ARG
+
+
+def test_estimate_mask_rejects(L):
+    args = lambda d=64, block=128, samples=16, tau=0.9, ws=None, wsb=0: (
+        FAKE, FAKE, 1, 2, 1024, d, block, samples, ctypes.c_float(tau), ws, wsb,
+        FAKE, FAKE, FAKE, None, None, None)
+    assert L.asa_estimate_mask(*args(d=80)) == asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_estimate_mask(*args(block=64)) == asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_estimate_mask(*args(samples=8)) == asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_estimate_mask(*args(tau=0.0)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_estimate_mask(*args(tau=float("nan"))) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_estimate_mask(*args()) == asa.ASA_ERR_WORKSPACE          # no workspace
+    assert L.asa_estimate_mask(*args(ws=ctypes.c_void_p(0x10010), wsb=1 << 30)) == \
+        asa.ASA_ERR_WORKSPACE                                               # not 256-aligned
+    need = L.asa_estimate_mask_workspace_size(1, 2, 1024)
+    assert need > 0
+    assert L.asa_estimate_mask(*args(ws=ctypes.c_void_p(0x100000), wsb=need - 1)) == \
+        asa.ASA_ERR_WORKSPACE
+    # one transposed pointer without the other
+    bad = list(args(ws=ctypes.c_void_p(0x100000), wsb=need))
+    bad[14] = FAKE
+    assert L.asa_estimate_mask(*bad) == asa.ASA_ERR_INVALID_ARG
+    # N too large, B*H too large
+    assert L.asa_estimate(FAKE, FAKE, 1, 1, 300000, 64, 128, 16, None, 0, FAKE, None) == \
+        asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_estimate(FAKE, FAKE, 300, 300, 1024, 64, 128, 16, None, 0, FAKE, None) == \
+        asa.ASA_ERR_UNSUPPORTED
+
+
+def test_attention_rejects(L):
+    assert L.asa_sparse_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 96, 128, 0, None, 0,
+                                 FAKE, FAKE, None) == asa.ASA_ERR_UNSUPPORTED
+    assert L.asa_sparse_attn_fwd(FAKE, FAKE, MIS, FAKE, FAKE, 1, 2, 1024, 64, 128, 0, None, 0,
+                                 FAKE, FAKE, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_sparse_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 64, 128, 64, None, 0,
+                                 FAKE, FAKE, None) == asa.ASA_ERR_WORKSPACE
+    assert L.asa_sparse_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 64, 128, -1, None, 0,
+                                 FAKE, FAKE, None) == asa.ASA_ERR_INVALID_ARG
+    args = [FAKE] * 10 + [1, 2, 1024, 64, 128, None, 0] + [FAKE] * 3 + [None]
+    assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_WORKSPACE
+    args[9] = None   # row_idx_t
+    assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(L):
+    nb = 256
+    est = L.asa_estimate_mask_workspace_size(1, 12, 32760)
+    assert est >= 12 * nb * nb * (16 * 4 + 4 + 1)
+    assert L.asa_fwd_workspace_size(1, 12, 32760, 128, 0) == 0
+    assert L.asa_fwd_workspace_size(1, 12, 32760, 128, 64) >= 2 * 12 * 512 * 128 * 2
+    assert L.asa_bwd_workspace_size(1, 12, 32760, 128) >= 2 * 12 * 32760 * 4
+    assert L.asa_estimate_mask_workspace_size(0, 12, 32760) == 0

@@ -1,0 +1,195 @@
+"""GPU parity: every step of the CUDA path (through the C ABI) against the fp64 oracle
+on the same seeded inputs, at sizes the oracle finishes in seconds that still span
+several blocks and a ragged tail, plus the degenerate cases.
+
+Bars: permutations and CSR masks bit-exact (mask rows may differ only where the
+oracle marks the row marginal); outputs and gradients max-abs <= 2e-2 and rel-L2 <=
+5e-3 against the oracle using the oracle's mask; LSE within 1e-3."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from inputs import WORKLOADS, make_inputs
+from video_dit_dynamic_gilbert_b200 import asa
+from gpu_util import (LSE_ABS, check_close, check_transposed, compare_masks, f64, mask_from_csr,
+                      upload_mask)
+
+pytestmark = pytest.mark.gpu
+
+BASE = WORKLOADS["tiny"]
+CASES = {
+    "tiny": BASE,
+    "one-ragged-block": BASE.with_(name="r105", B=2, H=3, d=128, T=3, Hg=5, W=7, seed=11),
+    "tail-lt-k": BASE.with_(name="r394", B=1, H=2, d=64, T=1, Hg=2, W=197, seed=12),
+    "d128-ragged": BASE.with_(name="r495", B=1, H=2, d=128, T=5, Hg=9, W=11, seed=13, tau=0.95),
+    "d64-b2": BASE.with_(name="r1200", B=2, H=2, d=64, T=6, Hg=10, W=20, seed=14),
+    "multi-tile": BASE.with_(name="r3072", B=1, H=4, d=128, T=8, Hg=16, W=24, seed=15, tau=0.95),
+}
+
+_cache = {}
+
+
+def setup_case(name):
+    """Seeded inputs, the oracle's permuted tensors, P_imp and mask (cached)."""
+    if name in _cache:
+        return _cache[name]
+    wl = CASES[name]
+    x = make_inputs(wl, with_dout=True)
+    perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
+    ref = {k: oracle.permute(f64(x[k]), perm) for k in ("q", "k", "v", "dout")}
+    pimp = oracle.estimate_pimp(ref["q"], ref["k"])
+    mask = oracle.build_mask(pimp, wl.tau)
+    marg = oracle.marginal_rows(pimp, wl.tau)
+    dev = {k: x[k].cuda() for k in ("q", "k", "v", "dout")}
+    _cache[name] = (wl, x, perm, ref, pimp, mask, marg, dev)
+    return _cache[name]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_permute_bit_exact(name):
+    wl, x, perm, ref, *_ , dev = setup_case(name)
+    qp, kp, vp = asa.asa_gilbert_permute3(dev["q"], dev["k"], dev["v"], wl.T, wl.Hg, wl.W)
+    for t, k in ((qp, "q"), (kp, "k"), (vp, "v")):
+        assert np.array_equal(f64(t), ref[k]), k
+    single = asa.asa_gilbert_permute(dev["dout"], wl.T, wl.Hg, wl.W)
+    assert np.array_equal(f64(single), ref["dout"])
+    back = asa.asa_unpermute(qp, wl.T, wl.Hg, wl.W)
+    assert torch.equal(back, dev["q"])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_estimate_matches_oracle(name):
+    wl, x, perm, ref, pimp, *_ , dev = setup_case(name)
+    qp = torch.from_numpy(ref["q"]).to(torch.bfloat16).cuda()
+    kp = torch.from_numpy(ref["k"]).to(torch.bfloat16).cuda()
+    got = f64(asa.asa_estimate(qp, kp))
+    np.testing.assert_allclose(got, pimp, rtol=2e-4, atol=1e-9)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("tau", [None, 0.5, 0.8, 0.99, 1.0, 1e-6])
+def test_mask_bit_exact(name, tau):
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    if tau is not None:
+        mask = oracle.build_mask(pimp, tau)
+        marg = oracle.marginal_rows(pimp, tau)
+    t = wl.tau if tau is None else tau
+    qp = torch.from_numpy(ref["q"]).to(torch.bfloat16).cuda()
+    kp = torch.from_numpy(ref["k"]).to(torch.bfloat16).cuda()
+    bm = asa.asa_estimate_mask(qp, kp, t, transposed=True)
+    gm = mask_from_csr(bm)
+    compare_masks(gm, mask, marg)
+    assert int(bm.nnz.item()) == int(gm.sum())
+    check_transposed(bm, gm)
+    if t >= 1.0:
+        assert gm.all()
+    # the same mask from the two-call path (P_imp, then the mask)
+    p = asa.asa_estimate(qp, kp)
+    bm2 = asa.asa_build_mask(p, wl.N, t)
+    assert np.array_equal(mask_from_csr(bm2), gm)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_with_oracle_mask(name):
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    O_ref, L_ref = oracle.asa_forward(ref["q"], ref["k"], ref["v"], mask)
+    qp, kp, vp = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda() for k in ("q", "k", "v"))
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, upload_mask(mask, wl.N))
+    check_close(f64(o), O_ref, what="O")
+    check_close(f64(lse), L_ref, max_abs=LSE_ABS, rel_l2=1e-4, what="LSE")
+
+
+@pytest.mark.parametrize("name", ["tiny", "d128-ragged", "tail-lt-k"])
+def test_forward_dense_tau_one(name):
+    wl, x, perm, ref, *_ = setup_case(name)
+    nb = -(-wl.N // 128)
+    full = np.ones((wl.B, wl.H, nb, nb), dtype=bool)
+    O_ref, L_ref = oracle.asa_forward(ref["q"], ref["k"], ref["v"], full)
+    qp, kp, vp = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda() for k in ("q", "k", "v"))
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, upload_mask(full, wl.N))
+    check_close(f64(o), O_ref, what="O dense")
+    check_close(f64(lse), L_ref, max_abs=LSE_ABS, rel_l2=1e-4, what="LSE dense")
+    # and the library's own tau = 1 mask is all blocks
+    bm = asa.asa_estimate_mask(qp, kp, 1.0)
+    assert mask_from_csr(bm).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "one-ragged-block", "d128-ragged", "d64-b2"])
+@pytest.mark.parametrize("n", [64, 16, 1, 200])
+def test_asa_g_forward(name, n):
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    O_ref, L_ref = oracle.asa_forward(ref["q"], ref["k"], ref["v"], mask, global_window=n)
+    qp, kp, vp = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda() for k in ("q", "k", "v"))
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, upload_mask(mask, wl.N), global_window=n)
+    check_close(f64(o), O_ref, what=f"O ASA_G n={n}")
+    check_close(f64(lse), L_ref, max_abs=LSE_ABS, rel_l2=1e-4, what="LSE ASA_G")
+
+
+@pytest.mark.parametrize("name", ["tiny", "one-ragged-block", "tail-lt-k"])
+@pytest.mark.parametrize("n", [64, 7, 1])
+def test_global_pool(name, n):
+    wl, x, perm, ref, *_ = setup_case(name)
+    kp = torch.from_numpy(ref["k"]).to(torch.bfloat16).cuda()
+    got = f64(asa.asa_global_pool(kp, n))
+    for bb in range(wl.B):
+        for h in range(wl.H):
+            exp = oracle.global_tokens(ref["k"][bb, h], n)
+            # fp32 vs fp64 mean: at most one bf16 rounding step apart
+            np.testing.assert_allclose(got[bb, h], exp, rtol=2 ** -7, atol=1e-6)
+            assert (got[bb, h] == exp).mean() > 0.99
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_with_oracle_mask(name):
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    dq_d, dkv_d = oracle.asa_backward(ref["q"], ref["k"], ref["v"], ref["dout"], mask)
+    qp, kp, vp, dop = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda()
+                       for k in ("q", "k", "v", "dout"))
+    bm = upload_mask(mask, wl.N)
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
+    dq, dk, dv = (f64(t) for t in asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm))
+    rq, rk, rv = np.zeros_like(dq), np.zeros_like(dk), np.zeros_like(dv)
+    for (bb, h, I), blk in dq_d.items():
+        rq[bb, h, 128 * I:128 * I + blk.shape[0]] = blk
+    for (bb, h, J), (gk, gv) in dkv_d.items():
+        rk[bb, h, 128 * J:128 * J + gk.shape[0]] = gk
+        rv[bb, h, 128 * J:128 * J + gv.shape[0]] = gv
+    check_close(dq, rq, what="dQ")
+    check_close(dk, rk, what="dK")
+    check_close(dv, rv, what="dV")
+
+
+@pytest.mark.parametrize("name", ["tiny", "d64-b2", "multi-tile"])
+def test_end_to_end_call(name):
+    """Raster q, k, v -> permute -> estimate + mask -> forward -> unpermute."""
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    out, lse, bm = asa.asa_attention(dev["q"], dev["k"], dev["v"], wl.T, wl.Hg, wl.W, wl.tau)
+    gm = mask_from_csr(bm)
+    compare_masks(gm, mask, marg)
+    O_ref, _ = oracle.asa_forward(ref["q"], ref["k"], ref["v"], mask)
+    # query blocks whose (marginal) mask row differs are left out of the comparison
+    agree = ~(gm != mask).any(axis=-1)                       # [B, H, nb]
+    got = f64(out)                                           # raster [B, N, H, d]
+    for bb in range(wl.B):
+        for h in range(wl.H):
+            rows = np.nonzero(np.repeat(agree[bb, h], 128)[:wl.N])[0]
+            check_close(got[bb, perm[rows], h], O_ref[bb, h, rows], what="O end-to-end")
+    asa.asa_check_device_status()
+
+
+def test_single_token_grid():
+    wl = BASE.with_(name="one", B=1, H=2, d=64, T=1, Hg=1, W=1, seed=21)
+    x = make_inputs(wl)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    out, lse, bm = asa.asa_attention(q, k, v, 1, 1, 1, 0.9)
+    assert mask_from_csr(bm).all()
+    torch.testing.assert_close(out.float(), v.float(), rtol=0, atol=1e-2)
+    ref_lse = (f64(q) * f64(k)).sum(-1)[0, 0] / math.sqrt(64)
+    np.testing.assert_allclose(f64(lse)[0, :, 0], ref_lse, atol=LSE_ABS)
+
+
+def test_device_status_ok():
+    asa.asa_check_device_status()

@@ -1,0 +1,297 @@
+"""Thin Python binding of libasa.so (include/asa.h), same names as the C ABI.
+
+Marshalling only: every step of the hot path runs in the library's CUDA kernels.
+PyTorch provides device memory (outputs, workspaces) and the current stream.
+There is no CPU fallback: a missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libasa.so")
+
+ASA_OK = 0
+ASA_ERR_INVALID_ARG = -1
+ASA_ERR_UNSUPPORTED = -2
+ASA_ERR_WORKSPACE = -3
+ASA_ERR_CUDA = -4
+ASA_ERR_TIMEOUT = -5
+BLOCK = 128
+SAMPLES = 16
+
+_c_int, _c_size, _c_float, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
+_SIGNATURES = {
+    "asa_version": ([], _c_int),
+    "asa_last_error_string": ([], ctypes.c_char_p),
+    "asa_gilbert_index": ([_c_int, _c_int, _c_int, _vp], _c_int),
+    "asa_gilbert_permute": ([_vp, _vp] + [_c_int] * 6 + [_vp], _c_int),
+    "asa_gilbert_permute3": ([_vp] * 6 + [_c_int] * 6 + [_vp], _c_int),
+    "asa_unpermute": ([_vp, _vp] + [_c_int] * 6 + [_vp], _c_int),
+    "asa_estimate_mask_workspace_size": ([_c_int] * 3, _c_size),
+    "asa_estimate": ([_vp, _vp] + [_c_int] * 6 + [_vp, _c_size, _vp, _vp], _c_int),
+    "asa_build_mask": ([_vp, _c_int, _c_int, _c_int, _c_float, _vp, _c_size] + [_vp] * 6, _c_int),
+    "asa_estimate_mask": ([_vp, _vp] + [_c_int] * 6 + [_c_float, _vp, _c_size] + [_vp] * 6, _c_int),
+    "asa_global_pool": ([_vp, _vp] + [_c_int] * 5 + [_vp], _c_int),
+    "asa_fwd_workspace_size": ([_c_int] * 5, _c_size),
+    "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
+    "asa_bwd_workspace_size": ([_c_int] * 4, _c_size),
+    "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 5 + [_vp, _c_size] + [_vp] * 4, _c_int),
+    "asa_check_device_status": ([_vp], _c_int),
+    "asa_shutdown": ([], None),
+}
+
+_lib = None
+
+
+class AsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"ASA error {code}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libasa.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m video_dit_dynamic_gilbert_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != ASA_OK:
+        raise AsaError(rc, lib().asa_last_error_string().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bf16_cuda(name: str, t: torch.Tensor, ndim: int = 4) -> None:
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == ndim):
+        raise ValueError(f"{name} must be a contiguous {ndim}-D bf16 CUDA tensor")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def nblocks(N: int) -> int:
+    return -(-N // BLOCK)
+
+
+# ----------------------------------------------------------------------- Preprocessing
+
+def asa_gilbert_index(T: int, Hg: int, W: int) -> np.ndarray:
+    """Host Gilbert table: perm[i] = raster index of curve position i."""
+    out = np.empty(T * Hg * W, dtype=np.int32)
+    _check(lib().asa_gilbert_index(T, Hg, W, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def asa_gilbert_permute(x: torch.Tensor, T: int, Hg: int, W: int, out=None, stream=None):
+    """x [B, N, H, d] raster -> xp [B, H, N, d] Gilbert order."""
+    _bf16_cuda("x", x)
+    B, N, H, d = x.shape
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=x.dtype, device=x.device)
+    _check(lib().asa_gilbert_permute(_ptr(x), _ptr(out), B, T, Hg, W, H, d, _stream(stream)))
+    return out
+
+
+def asa_gilbert_permute3(q, k, v, T: int, Hg: int, W: int, outs=None, stream=None):
+    for n_, t in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n_, t)
+    B, N, H, d = q.shape
+    if outs is None:
+        outs = tuple(torch.empty((B, H, N, d), dtype=q.dtype, device=q.device) for _ in range(3))
+    _check(lib().asa_gilbert_permute3(_ptr(q), _ptr(k), _ptr(v), *(_ptr(o) for o in outs),
+                                      B, T, Hg, W, H, d, _stream(stream)))
+    return outs
+
+
+def asa_unpermute(xp: torch.Tensor, T: int, Hg: int, W: int, out=None, stream=None):
+    """xp [B, H, N, d] Gilbert order -> x [B, N, H, d] raster."""
+    _bf16_cuda("xp", xp)
+    B, H, N, d = xp.shape
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=xp.dtype, device=xp.device)
+    _check(lib().asa_unpermute(_ptr(xp), _ptr(out), B, T, Hg, W, H, d, _stream(stream)))
+    return out
+
+
+# ----------------------------------------------------------------------- Steps 1, 2.1
+
+@dataclass
+class BlockMask:
+    """CSR of kept key blocks per query block (and its transpose), device int32."""
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    nnz: torch.Tensor
+    col_ptr_t: torch.Tensor | None
+    row_idx_t: torch.Tensor | None
+    B: int
+    H: int
+    N: int
+
+    @property
+    def nb(self) -> int:
+        return nblocks(self.N)
+
+
+def estimate_mask_workspace(B: int, H: int, N: int, device) -> torch.Tensor:
+    return _workspace(lib().asa_estimate_mask_workspace_size(B, H, N), device)
+
+
+def _alloc_mask(B, H, N, device, transposed):
+    nb = nblocks(N)
+    rows = B * H * nb
+    cap = rows * nb
+    z = dict(dtype=torch.int32, device=device)
+    return BlockMask(torch.empty(rows + 1, **z), torch.empty(max(cap, 1), **z), torch.empty(1, **z),
+                     torch.empty(rows + 1, **z) if transposed else None,
+                     torch.empty(max(cap, 1), **z) if transposed else None, B, H, N)
+
+
+def asa_estimate(qp: torch.Tensor, kp: torch.Tensor, workspace=None, out=None, stream=None):
+    """P_imp [B, H, nb, nb] fp32 from the sampled tokens (Step 1)."""
+    _bf16_cuda("qp", qp)
+    _bf16_cuda("kp", kp)
+    B, H, N, d = qp.shape
+    nb = nblocks(N)
+    if workspace is None:
+        workspace = estimate_mask_workspace(B, H, N, qp.device)
+    if out is None:
+        out = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qp.device)
+    _check(lib().asa_estimate(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, _ptr(workspace),
+                              workspace.numel(), _ptr(out), _stream(stream)))
+    return out
+
+
+def asa_build_mask(p_imp: torch.Tensor, N: int, tau: float, transposed: bool = True,
+                   workspace=None, mask: BlockMask | None = None, stream=None) -> BlockMask:
+    """Kept-block CSR from P_imp (Step 2.1)."""
+    if not (p_imp.is_cuda and p_imp.dtype == torch.float32 and p_imp.is_contiguous()):
+        raise ValueError("p_imp must be a contiguous fp32 CUDA tensor")
+    B, H = p_imp.shape[:2]
+    if workspace is None:
+        workspace = estimate_mask_workspace(B, H, N, p_imp.device)
+    m = mask or _alloc_mask(B, H, N, p_imp.device, transposed)
+    _check(lib().asa_build_mask(_ptr(p_imp), B, H, N, float(tau), _ptr(workspace), workspace.numel(),
+                                _ptr(m.row_ptr), _ptr(m.col_idx), _ptr(m.nnz), _ptr(m.col_ptr_t),
+                                _ptr(m.row_idx_t), _stream(stream)))
+    return m
+
+
+def asa_estimate_mask(qp: torch.Tensor, kp: torch.Tensor, tau: float, transposed: bool = True,
+                      workspace=None, mask: BlockMask | None = None, stream=None) -> BlockMask:
+    """Steps 1 + 2.1 in one call."""
+    _bf16_cuda("qp", qp)
+    _bf16_cuda("kp", kp)
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = estimate_mask_workspace(B, H, N, qp.device)
+    m = mask or _alloc_mask(B, H, N, qp.device, transposed)
+    _check(lib().asa_estimate_mask(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, float(tau),
+                                   _ptr(workspace), workspace.numel(), _ptr(m.row_ptr),
+                                   _ptr(m.col_idx), _ptr(m.nnz), _ptr(m.col_ptr_t),
+                                   _ptr(m.row_idx_t), _stream(stream)))
+    return m
+
+
+# ----------------------------------------------------------------------- Step 2.2
+
+def asa_global_pool(xp: torch.Tensor, n: int, out=None, stream=None):
+    _bf16_cuda("xp", xp)
+    B, H, N, d = xp.shape
+    G = -(-N // n)
+    if out is None:
+        out = torch.empty((B, H, G, d), dtype=xp.dtype, device=xp.device)
+    _check(lib().asa_global_pool(_ptr(xp), _ptr(out), B, H, N, d, n, _stream(stream)))
+    return out
+
+
+def fwd_workspace(B, H, N, d, global_window, device):
+    return _workspace(lib().asa_fwd_workspace_size(B, H, N, d, global_window), device)
+
+
+def asa_sparse_attn_fwd(qp, kp, vp, mask: BlockMask, global_window: int = 0, workspace=None,
+                        out=None, lse=None, stream=None):
+    """O [B, H, N, d] bf16 and natural-log LSE [B, H, N] fp32 over the kept tiles."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp)):
+        _bf16_cuda(n_, t)
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = fwd_workspace(B, H, N, d, global_window, qp.device)
+    if out is None:
+        out = torch.empty_like(qp)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=qp.device)
+    _check(lib().asa_sparse_attn_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(mask.row_ptr),
+                                     _ptr(mask.col_idx), B, H, N, d, BLOCK, global_window,
+                                     _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                     _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def bwd_workspace(B, H, N, d, device):
+    return _workspace(lib().asa_bwd_workspace_size(B, H, N, d), device)
+
+
+def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, workspace=None, outs=None,
+                        stream=None):
+    """dQ, dK, dV [B, H, N, d] bf16 under the fixed mask (standard ASA)."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp), ("o", o), ("dout", dout)):
+        _bf16_cuda(n_, t)
+    if mask.col_ptr_t is None:
+        raise ValueError("the backward needs the transposed CSR (transposed=True)")
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = bwd_workspace(B, H, N, d, qp.device)
+    if outs is None:
+        outs = tuple(torch.empty_like(qp) for _ in range(3))
+    _check(lib().asa_sparse_attn_bwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(o), _ptr(dout), _ptr(lse),
+                                     _ptr(mask.row_ptr), _ptr(mask.col_idx), _ptr(mask.col_ptr_t),
+                                     _ptr(mask.row_idx_t), B, H, N, d, BLOCK, _ptr(workspace),
+                                     workspace.numel(), *(_ptr(t) for t in outs), _stream(stream)))
+    return outs
+
+
+def asa_check_device_status(stream=None) -> None:
+    _check(lib().asa_check_device_status(_stream(stream)))
+
+
+def asa_shutdown() -> None:
+    lib().asa_shutdown()
+
+
+# ----------------------------------------------------------------------- one attention call
+
+def asa_attention(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
+                  stream=None):
+    """One ASA self-attention call on raster-layout q, k, v [B, N, H, d]: Gilbert permute,
+    estimate + mask, block-sparse forward, unpermute.  Returns (O raster, LSE, mask)."""
+    qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W, stream=stream)
+    mask = asa_estimate_mask(qp, kp, tau, transposed=False, stream=stream)
+    op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window, stream=stream)
+    return asa_unpermute(op, T, Hg, W, stream=stream), lse, mask

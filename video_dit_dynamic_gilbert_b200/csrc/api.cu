@@ -1,0 +1,423 @@
+// C ABI of libasa.so (declarations and contracts in include/asa.h).
+//
+// Every entry point validates its arguments on the host before it launches
+// anything, carves the caller's workspace, and launches the kernels of its step on
+// the caller's stream.  The only memory the library owns is the per-shape Gilbert
+// permutation table (built on the host once per (device, T, Hg, W) and uploaded).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/asa.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(ASA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int num_sms_current() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+std::mutex g_perm_mu;
+std::map<std::tuple<int, int, int, int>, int32_t*> g_perm_cache;
+
+// Device copy of the Gilbert table for the current device (built once per shape).
+int get_perm(int T, int Hg, int W, const int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_perm_mu);
+  auto key = std::make_tuple(dev, T, Hg, W);
+  auto it = g_perm_cache.find(key);
+  if (it != g_perm_cache.end()) {
+    *out = it->second;
+    return ASA_OK;
+  }
+  const size_t N = static_cast<size_t>(T) * Hg * W;
+  std::vector<int32_t> host(N);
+  if (!asa::gilbert_order_host(T, Hg, W, host.data()))
+    return fail(ASA_ERR_INVALID_ARG, "gilbert order failed for %dx%dx%d", T, Hg, W);
+  int32_t* d = nullptr;
+  e = cudaMalloc(&d, N * sizeof(int32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(permutation table)");
+  e = cudaMemcpy(d, host.data(), N * sizeof(int32_t), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(d);
+    return cuda_fail(e, "cudaMemcpy(permutation table)");
+  }
+  g_perm_cache[key] = d;
+  *out = d;
+  return ASA_OK;
+}
+
+int check_common(int B, int H, int N, int d) {
+  if (B < 1 || H < 1) return fail(ASA_ERR_INVALID_ARG, "B=%d and H=%d must be >= 1", B, H);
+  if (static_cast<int64_t>(B) * H > 65535)
+    return fail(ASA_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", static_cast<long long>(B) * H);
+  if (N < 1) return fail(ASA_ERR_INVALID_ARG, "N=%d must be >= 1", N);
+  if (N > ASA_MAX_TOKENS) return fail(ASA_ERR_UNSUPPORTED, "N=%d exceeds %d", N, ASA_MAX_TOKENS);
+  if (d != 64 && d != 128) return fail(ASA_ERR_UNSUPPORTED, "head dim d=%d not in {64,128}", d);
+  return ASA_OK;
+}
+
+int check_grid(int T, int Hg, int W, int64_t* N) {
+  if (T < 1 || Hg < 1 || W < 1)
+    return fail(ASA_ERR_INVALID_ARG, "grid %dx%dx%d: sides must be >= 1", T, Hg, W);
+  const int64_t n = static_cast<int64_t>(T) * Hg * W;
+  if (n > ASA_MAX_TOKENS)
+    return fail(ASA_ERR_UNSUPPORTED, "grid %dx%dx%d has %lld > %d tokens", T, Hg, W,
+                static_cast<long long>(n), ASA_MAX_TOKENS);
+  *N = n;
+  return ASA_OK;
+}
+
+int check_ptr(const void* p, const char* name, bool need16 = true) {
+  if (p == nullptr) return fail(ASA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (need16 && !aligned16(p)) return fail(ASA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  if (!need16 && (reinterpret_cast<uintptr_t>(p) & 3u))
+    return fail(ASA_ERR_INVALID_ARG, "%s is not 4-byte aligned", name);
+  return ASA_OK;
+}
+
+#define ASA_TRY(x)          \
+  do {                      \
+    const int rc__ = (x);   \
+    if (rc__ != ASA_OK) return rc__; \
+  } while (0)
+
+struct MaskWs {
+  float* G;
+  float* lse2;
+  float* p_imp;
+  uint8_t* bitmap;
+  int32_t* counts;
+  int32_t* counts_t;
+  size_t bytes;
+};
+
+MaskWs carve_mask_ws(void* base, int BH, int nb) {
+  MaskWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off += align256(n);
+    return o;
+  };
+  const size_t o_g = take(asa::est_scratch_floats(BH, nb) * sizeof(float));
+  const size_t o_p = take(static_cast<size_t>(BH) * nb * nb * sizeof(float));
+  const size_t o_b = take(static_cast<size_t>(BH) * nb * nb);
+  const size_t o_c = take(static_cast<size_t>(BH) * nb * sizeof(int32_t));
+  const size_t o_t = take(static_cast<size_t>(BH) * nb * sizeof(int32_t));
+  w.bytes = off;
+  if (base) {
+    char* b = static_cast<char*>(base);
+    w.G = reinterpret_cast<float*>(b + o_g);
+    w.lse2 = w.G + static_cast<size_t>(BH) * nb * asa::kSamplesHost * nb;
+    w.p_imp = reinterpret_cast<float*>(b + o_p);
+    w.bitmap = reinterpret_cast<uint8_t*>(b + o_b);
+    w.counts = reinterpret_cast<int32_t*>(b + o_c);
+    w.counts_t = reinterpret_cast<int32_t*>(b + o_t);
+  }
+  return w;
+}
+
+int check_ws(const void* ws, size_t have, size_t need) {
+  if (need == 0) return ASA_OK;
+  if (ws == nullptr) return fail(ASA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(ASA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (have < need) return fail(ASA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", have, need);
+  return ASA_OK;
+}
+
+int check_block(int block, int samples) {
+  if (block != ASA_BLOCK) return fail(ASA_ERR_UNSUPPORTED, "block=%d (only 128)", block);
+  if (samples != ASA_SAMPLES) return fail(ASA_ERR_UNSUPPORTED, "samples=%d (only 16)", samples);
+  return ASA_OK;
+}
+
+}  // namespace
+
+__device__ unsigned int g_device_error = 0;
+
+extern "C" {
+
+int asa_version(void) { return 100; }
+
+const char* asa_last_error_string(void) { return g_last_error.c_str(); }
+
+int asa_gilbert_index(int T, int Hg, int W, int32_t* perm_host) {
+  int64_t N = 0;
+  ASA_TRY(check_grid(T, Hg, W, &N));
+  ASA_TRY(check_ptr(perm_host, "perm_host", false));
+  if (!asa::gilbert_order_host(T, Hg, W, perm_host))
+    return fail(ASA_ERR_INVALID_ARG, "gilbert order failed for %dx%dx%d", T, Hg, W);
+  return ASA_OK;
+}
+
+static int permute_impl(const void* const* src, void* const* dst, int nt, bool to_perm, int B,
+                        int T, int Hg, int W, int H, int d, void* stream) {
+  int64_t N = 0;
+  ASA_TRY(check_grid(T, Hg, W, &N));
+  ASA_TRY(check_common(B, H, static_cast<int>(N), d));
+  for (int k = 0; k < nt; ++k) {
+    ASA_TRY(check_ptr(src[k], "input"));
+    ASA_TRY(check_ptr(dst[k], "output"));
+    if (src[k] == dst[k]) return fail(ASA_ERR_INVALID_ARG, "input and output alias");
+  }
+  const int32_t* perm = nullptr;
+  ASA_TRY(get_perm(T, Hg, W, &perm));
+  cudaError_t e = asa::launch_permute(src, dst, nt, to_perm, perm, B, static_cast<int>(N), H, d,
+                                      num_sms_current(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, to_perm ? "permute launch" : "unpermute launch");
+  return ASA_OK;
+}
+
+int asa_gilbert_permute(const void* x, void* xp, int B, int T, int Hg, int W, int H, int d,
+                        void* stream) {
+  const void* s[1] = {x};
+  void* t[1] = {xp};
+  return permute_impl(s, t, 1, true, B, T, Hg, W, H, d, stream);
+}
+
+int asa_gilbert_permute3(const void* x0, const void* x1, const void* x2, void* xp0, void* xp1,
+                         void* xp2, int B, int T, int Hg, int W, int H, int d, void* stream) {
+  const void* s[3] = {x0, x1, x2};
+  void* t[3] = {xp0, xp1, xp2};
+  return permute_impl(s, t, 3, true, B, T, Hg, W, H, d, stream);
+}
+
+int asa_unpermute(const void* xp, void* x, int B, int T, int Hg, int W, int H, int d, void* stream) {
+  const void* s[1] = {xp};
+  void* t[1] = {x};
+  return permute_impl(s, t, 1, false, B, T, Hg, W, H, d, stream);
+}
+
+size_t asa_estimate_mask_workspace_size(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1 || N > ASA_MAX_TOKENS) return 0;
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  return carve_mask_ws(nullptr, B * H, nb).bytes;
+}
+
+int asa_estimate(const void* qp, const void* kp, int B, int H, int N, int d, int block, int samples,
+                 void* workspace, size_t ws_bytes, float* p_imp, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, samples));
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(p_imp, "p_imp", false));
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  MaskWs w = carve_mask_ws(workspace, B * H, nb);
+  ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
+  cudaError_t e = asa::launch_estimate(qp, kp, B * H, N, d, w.G, w.lse2, p_imp, num_sms_current(),
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
+  return ASA_OK;
+}
+
+static int build_mask_impl(const float* p_imp, int B, int H, int N, float tau, const MaskWs& w,
+                           int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                           int32_t* col_ptr_t, int32_t* row_idx_t, void* stream) {
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  cudaError_t e = asa::launch_build_mask(p_imp, B * H, nb, tau, w.bitmap, w.counts, row_ptr, col_idx,
+                                         nnz_out, w.counts_t, col_ptr_t, row_idx_t,
+                                         num_sms_current(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
+  return ASA_OK;
+}
+
+static int check_mask_args(float tau, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                           int32_t* col_ptr_t, int32_t* row_idx_t) {
+  if (!(tau > 0.f)) return fail(ASA_ERR_INVALID_ARG, "tau=%g must be > 0", static_cast<double>(tau));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(nnz_out, "nnz_out", false));
+  if ((col_ptr_t == nullptr) != (row_idx_t == nullptr))
+    return fail(ASA_ERR_INVALID_ARG, "col_ptr_t and row_idx_t must both be set or both NULL");
+  if (col_ptr_t) {
+    ASA_TRY(check_ptr(col_ptr_t, "col_ptr_t", false));
+    ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
+  }
+  return ASA_OK;
+}
+
+int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* workspace,
+                   size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                   int32_t* col_ptr_t, int32_t* row_idx_t, void* stream) {
+  ASA_TRY(check_common(B, H, N, 64));
+  ASA_TRY(check_ptr(p_imp, "p_imp", false));
+  ASA_TRY(check_mask_args(tau, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t));
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  MaskWs w = carve_mask_ws(workspace, B * H, nb);
+  ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
+  return build_mask_impl(p_imp, B, H, N, tau, w, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t,
+                         stream);
+}
+
+int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d, int block,
+                      int samples, float tau, void* workspace, size_t ws_bytes, int32_t* row_ptr,
+                      int32_t* col_idx, int32_t* nnz_out, int32_t* col_ptr_t, int32_t* row_idx_t,
+                      void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, samples));
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_mask_args(tau, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t));
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  MaskWs w = carve_mask_ws(workspace, B * H, nb);
+  ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
+  cudaError_t e = asa::launch_estimate(qp, kp, B * H, N, d, w.G, w.lse2, w.p_imp, num_sms_current(),
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
+  return build_mask_impl(w.p_imp, B, H, N, tau, w, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t,
+                         stream);
+}
+
+int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_ptr(xp, "xp"));
+  ASA_TRY(check_ptr(xg, "xg"));
+  if (n < 1) return fail(ASA_ERR_INVALID_ARG, "global window n=%d must be >= 1", n);
+  cudaError_t e = asa::launch_global_pool(xp, xg, B * H, N, d, n, num_sms_current(),
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+  return ASA_OK;
+}
+
+size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window) {
+  if (global_window <= 0 || B < 1 || H < 1 || N < 1) return 0;
+  const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+  return 2 * align256(static_cast<size_t>(B) * H * G * d * 2);
+}
+
+int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                        const int32_t* col_idx, int B, int H, int N, int d, int block,
+                        int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
+                        void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(vp, "vp"));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(o, "o"));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  const size_t need = asa_fwd_workspace_size(B, H, N, d, global_window);
+  ASA_TRY(check_ws(workspace, ws_bytes, need));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* kg = nullptr;
+  const void* vg = nullptr;
+  if (global_window > 0) {
+    const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    char* base = static_cast<char*>(workspace);
+    void* kgw = base;
+    void* vgw = base + align256(static_cast<size_t>(B) * H * G * d * 2);
+    cudaError_t e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, num_sms_current(), s);
+    if (e == cudaSuccess)
+      e = asa::launch_global_pool(vp, vgw, B * H, N, d, global_window, num_sms_current(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    kg = kgw;
+    vg = vgw;
+  }
+  cudaError_t e = asa::launch_fwd_mma(qp, kp, vp, row_ptr, col_idx, kg, vg, B * H, N, d,
+                                      global_window, o, lse, s);
+  if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return ASA_OK;
+}
+
+size_t asa_bwd_workspace_size(int B, int H, int N, int d) {
+  (void)d;
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return 2 * align256(static_cast<size_t>(B) * H * N * sizeof(float));
+}
+
+int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
+                        const void* dout, const float* lse, const int32_t* row_ptr,
+                        const int32_t* col_idx, const int32_t* col_ptr_t,
+                        const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                        void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
+                        void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  const void* bf[] = {qp, kp, vp, o, dout, dq, dk, dv};
+  const char* names[] = {"qp", "kp", "vp", "o", "dout", "dq", "dk", "dv"};
+  for (int k = 0; k < 8; ++k) ASA_TRY(check_ptr(bf[k], names[k]));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(col_ptr_t, "col_ptr_t", false));
+  ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
+  const size_t need = asa_bwd_workspace_size(B, H, N, d);
+  ASA_TRY(check_ws(workspace, ws_bytes, need));
+  float* Dvec = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         align256(static_cast<size_t>(B) * H * N * sizeof(float)));
+  cudaError_t e = asa::launch_bwd_mma(qp, kp, vp, o, dout, lse, row_ptr, col_idx, col_ptr_t,
+                                      row_idx_t, B * H, N, d, Dvec, lse2, dq, dk, dv,
+                                      num_sms_current(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return ASA_OK;
+}
+
+int asa_check_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    return fail(ASA_ERR_TIMEOUT, "a device-side bounded wait expired (word 0x%x)", word);
+  }
+  return ASA_OK;
+}
+
+void asa_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_perm_mu);
+  int cur = 0;
+  const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+  for (auto& kv : g_perm_cache) {
+    if (have_dev) cudaSetDevice(std::get<0>(kv.first));
+    cudaFree(kv.second);
+  }
+  if (have_dev) cudaSetDevice(cur);
+  g_perm_cache.clear();
+}
+
+}  // extern "C"

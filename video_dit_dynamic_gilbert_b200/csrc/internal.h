@@ -1,0 +1,41 @@
+// Launchers shared between the kernel files and the C ABI (api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace asa {
+
+constexpr int kSamplesHost = 16;  // k: sampled tokens per block
+
+bool gilbert_order_host(int T, int Hg, int W, int32_t* out);
+
+cudaError_t launch_permute(const void* const* src, void* const* dst, int ntensors, bool to_permuted,
+                           const int32_t* perm_dev, int B, int N, int H, int d, int num_sms,
+                           cudaStream_t stream);
+
+size_t est_scratch_floats(int BH, int nb);
+cudaError_t launch_estimate(const void* qp, const void* kp, int BH, int N, int d, float* G,
+                            float* lse2, float* p_imp, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uint8_t* bitmap,
+                              int32_t* counts, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                              int32_t* counts_t, int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,
+                              cudaStream_t stream);
+
+cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, int n, int num_sms,
+                               cudaStream_t stream);
+
+cudaError_t launch_fwd_mma(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                           const int32_t* col_idx, const void* kg, const void* vg, int BH, int N,
+                           int d, int global_window, void* o, float* lse, cudaStream_t stream);
+
+cudaError_t launch_bwd_mma(const void* qp, const void* kp, const void* vp, const void* o,
+                           const void* dout, const float* lse, const int32_t* row_ptr,
+                           const int32_t* col_idx, const int32_t* col_ptr_t,
+                           const int32_t* row_idx_t, int BH, int N, int d, float* Dvec,
+                           float* lse2, void* dq, void* dk, void* dv, int num_sms,
+                           cudaStream_t stream);
+
+}  // namespace asa
