@@ -173,6 +173,17 @@ int check_block(int block, int samples) {
 
 __device__ unsigned int g_device_error = 0;
 
+namespace {
+// Device address of g_device_error for the current device (kernels set bits in it
+// when a bounded wait expires).
+cudaError_t device_error_word(unsigned int** out) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+  *out = static_cast<unsigned int*>(p);
+  return e;
+}
+}  // namespace
+
 extern "C" {
 
 int asa_version(void) { return 100; }
@@ -354,8 +365,11 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
     kg = kgw;
     vg = vgw;
   }
-  cudaError_t e = asa::launch_fwd_mma(qp, kp, vp, row_ptr, col_idx, kg, vg, B * H, N, d,
-                                      global_window, o, lse, s);
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_fwd_tc(qp, kp, vp, row_ptr, col_idx, kg, vg, B * H, N, d, global_window, o, lse,
+                         err_word, s);
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
   return ASA_OK;
 }

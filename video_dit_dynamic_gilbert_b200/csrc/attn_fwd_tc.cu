@@ -1,0 +1,414 @@
+// Block-sparse attention forward on tcgen05 tensor cores (Video-BLADE, "Step 2.2:
+// Computation": standard ASA over the kept tiles of M, and ASA_G with global tokens).
+//
+// One CTA per (b, h, query block I of 128 rows), 6 warps, warp-specialised:
+//   warp 0      TMA producer: Q once, then for every kept key block J (the CSR row
+//               of I) its 128-row K and V tiles into an NST-stage ring; for ASA_G
+//               then the ceil(N/n) global tokens in 128-row tiles.  Tiles past N
+//               (ragged last block) are zero-filled by TMA.
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_j = Q K_j^T   (SS MMA, M=128 N=128, into TMEM S buffer j%2)
+//                 O  += P_j V_j   (TS MMA: P read from TMEM, V from shared memory)
+//               S_{j+1} is issued before PV_j so it overlaps the softmax of tile j.
+//   warps 2..5  softmax warpgroup: thread = query row = TMEM lane.  Reads S_j,
+//               masks columns past the tile's valid rows, keeps the running max /
+//               sum in the log2 domain, writes P_j as bf16 over S_j in TMEM, and
+//               rescales O in TMEM only when the running max grows by more than
+//               2^8 (until then P is taken against the stale max; exact after the
+//               final division).  Epilogue: O / l -> bf16 rows, LSE (natural log).
+// TMEM: S buffers at columns [0,128) and [128,256), O at [256, 256+D).
+// Every wait is bounded: on expiry the kernel sets the device error word, drains its
+// own copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace asa {
+
+namespace {
+
+constexpr int kFwdTcThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D, int NST>
+struct FwdTcLayout {
+  static constexpr uint32_t kTile = 128u * D * 2u;  // one 128-row bf16 tile of Q, K or V
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + kTile;
+  static constexpr uint32_t kV = kK + NST * kTile;
+  static constexpr uint32_t kBars = kV + NST * kTile;
+  // barriers: q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2],
+  //           o_done, drain; then the TMEM base address slot
+  static constexpr uint32_t kNumBars = 1 + 3 * NST + 2 + 2 + 1 + 1;
+  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr uint32_t kBytes = kTmemSlot + 16;
+  static constexpr uint32_t kSmem = kBytes + 1024;  // + alignment slack
+};
+
+struct TileSrc {
+  int row0, nvalid;
+  bool global;
+};
+
+__device__ __forceinline__ TileSrc tile_src(int j, int nfine, const int32_t* cols, int N, int G) {
+  TileSrc t;
+  if (j < nfine) {
+    t.row0 = cols[j] * kBlock;
+    t.nvalid = min(kBlock, N - t.row0);
+    t.global = false;
+  } else {
+    t.row0 = (j - nfine) * kBlock;
+    t.nvalid = min(kBlock, G - t.row0);
+    t.global = true;
+  }
+  return t;
+}
+
+template <int D, int NST>
+__global__ void __launch_bounds__(kFwdTcThreads, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
+                  const __grid_constant__ CUtensorMap tmVg, const int32_t* __restrict__ row_ptr,
+                  const int32_t* __restrict__ col_idx, int N, int nb, int G, float gbias2,
+                  float c2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                  unsigned int* __restrict__ err_word, long long wait_limit) {
+  using L = FwdTcLayout<D, NST>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sbase = smem_raw + (base - raw);
+
+  const int I = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q0 = I * kBlock;
+  const int rbeg = row_ptr[bh * nb + I];
+  const int nfine = row_ptr[bh * nb + I + 1] - rbeg;
+  const int nglob = G > 0 ? (G + kBlock - 1) / kBlock : 0;
+  const int ntile = nfine + nglob;
+  const int32_t* cols = col_idx + rbeg;
+
+  const uint32_t bar0 = base + L::kBars;
+  auto q_full = [&]() { return bar0; };
+  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (1 + NST + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NST + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (1 + 3 * NST + b); };
+  auto p_full = [&](int b) { return bar0 + 8u * (3 + 3 * NST + b); };
+  const uint32_t o_done = bar0 + 8u * (5 + 3 * NST);
+  const uint32_t drain = bar0 + 8u * (6 + 3 * NST);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kTmemSlot);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full(), 1);
+    for (int s = 0; s < NST; ++s) {
+      tc::mbar_init(k_full(s), 1);
+      tc::mbar_init(v_full(s), 1);
+      tc::mbar_init(kv_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(s_full(b), 1);
+      tc::mbar_init(p_full(b), 128);
+    }
+    tc::mbar_init(o_done, 1);
+    tc::mbar_init(drain, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::tma_prefetch(&tmQ);
+      tc::tma_prefetch(&tmK);
+      tc::tma_prefetch(&tmV);
+      tc::mbar_expect_tx(q_full(), L::kTile);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tc::tma_load_3d(base + L::kQ + h * 16384u, &tmQ, 64 * h, q0, bh, q_full());
+      int issued = 0;
+      for (int j = 0; j < ntile; ++j) {
+        const int st = j % NST, n = j / NST;
+        if (n > 0 && !tc::mbar_wait(kv_empty(st), (n - 1) & 1, wait_limit)) {
+          failed = true;
+          break;
+        }
+        const TileSrc t = tile_src(j, nfine, cols, N, G);
+        const CUtensorMap* mk = t.global ? &tmKg : &tmK;
+        const CUtensorMap* mv = t.global ? &tmVg : &tmV;
+        tc::mbar_expect_tx(k_full(st), L::kTile);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tc::tma_load_3d(base + L::kK + st * L::kTile + h * 16384u, mk, 64 * h, t.row0, bh,
+                          k_full(st));
+        tc::mbar_expect_tx(v_full(st), L::kTile);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tc::tma_load_3d(base + L::kV + st * L::kTile + h * 16384u, mv, 64 * h, t.row0, bh,
+                          v_full(st));
+        issued = j + 1;
+      }
+      // drain: every issued copy has landed, and the MMAs have released the last
+      // stages (their commits arrive before the CTA exits)
+      tc::mbar_wait(q_full(), 0, wait_limit);
+      for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j) {
+        tc::mbar_wait(k_full(j % NST), (j / NST) & 1, wait_limit);
+        tc::mbar_wait(v_full(j % NST), (j / NST) & 1, wait_limit);
+        tc::mbar_wait(kv_empty(j % NST), (j / NST) & 1, wait_limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idPV = tc::idesc_bf16(128, D, false, true);
+      const uint32_t tO = tmem + 256u;
+      auto issue_s = [&](int j) {
+        const int st = j % NST;
+        const uint32_t dS = tmem + 128u * (j & 1);
+        const uint32_t kb = base + L::kK + st * L::kTile;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+          tc::umma_ss(dS, tc::sdesc_sw128(base + L::kQ + off, 16, 1024),
+                      tc::sdesc_sw128(kb + off, 16, 1024), idS, ks > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = tc::mbar_wait(q_full(), 0, wait_limit);
+      int issued_any = 0;
+      if (ok && ntile > 0) {
+        ok = tc::mbar_wait(k_full(0), 0, wait_limit);
+        if (ok) {
+          tc::fence_after();
+          issue_s(0);
+          tc::umma_commit(s_full(0));
+          issued_any = 1;
+        }
+      }
+      for (int j = 0; ok && j < ntile; ++j) {
+        if (j + 1 < ntile) {
+          const int st1 = (j + 1) % NST;
+          if (!(ok = tc::mbar_wait(k_full(st1), ((j + 1) / NST) & 1, wait_limit))) break;
+          tc::fence_after();
+          issue_s(j + 1);
+          tc::umma_commit(s_full((j + 1) & 1));
+        }
+        if (!(ok = tc::mbar_wait(p_full(j & 1), (j >> 1) & 1, wait_limit))) break;
+        if (!(ok = tc::mbar_wait(v_full(j % NST), (j / NST) & 1, wait_limit))) break;
+        tc::fence_after();
+        const uint32_t tP = tmem + 128u * (j & 1);
+        const uint32_t vb = base + L::kV + (j % NST) * L::kTile;
+#pragma unroll
+        for (int ks = 0; ks < kBlock / 16; ++ks)
+          tc::umma_ts(tO, tP + 8u * ks, tc::sdesc_sw128(vb + ks * 2048u, 16384, 1024), idPV,
+                      (j > 0 || ks > 0) ? 1u : 0u);
+        tc::umma_commit(kv_empty(j % NST));
+        tc::umma_commit(o_done);
+      }
+      failed = !ok;
+      if (issued_any) {
+        // drain: all MMAs of this CTA complete before TMEM is released
+        tc::umma_commit(drain);
+        tc::mbar_wait(drain, 0, wait_limit);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup
+    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      const bool ok = tc::mbar_wait(bar, parity, wait_limit);
+      return __all_sync(0xffffffffu, ok) != 0;
+    };
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < ntile; ++j) {
+      const int b = j & 1;
+      if (!wait_all(s_full(b), (j >> 1) & 1)) {
+        failed = true;
+        break;
+      }
+      tc::fence_after();
+      const TileSrc t = tile_src(j, nfine, cols, N, G);
+      const float bias = t.global ? gbias2 : 0.f;
+      uint32_t s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32_sync(trow + 128u * b + 32u * c, s + 32 * c);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; ++k) {
+        const float x = k < t.nvalid ? fmaf(__uint_as_float(s[k]), c2, bias) : -INFINITY;
+        s[k] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      if (j > 0) {
+        // PV_{j-1} done: O is stable (and the o_done phases stay in step)
+        if (!wait_all(o_done, (j - 1) & 1)) {
+          failed = true;
+          break;
+        }
+        tc::fence_after();
+      }
+      const bool need = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + 8.f);
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tc::tmem_ld32_sync(trow + 256u + 32u * c, ov);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+            tc::tmem_st16(trow + 256u + 32u * c, ov);
+            tc::tmem_st16(trow + 256u + 32u * c + 16u, ov + 16);
+            tc::tmem_wait_st();
+          }
+        }
+        if (need) m_ref = m_new;
+      }
+      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+      uint32_t p[64];
+      float rs = 0.f;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        const float a = fast_exp2(__uint_as_float(s[2 * k]) - mu);
+        const float bb = fast_exp2(__uint_as_float(s[2 * k + 1]) - mu);
+        rs += a + bb;
+        p[k] = pack_bf16(a, bb);
+      }
+      l += rs;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_st16(trow + 128u * b + 16u * c, p + 16 * c);
+      tc::tmem_wait_st();
+      tc::fence_before();
+      tc::mbar_arrive(p_full(b));
+    }
+    bool have_o = false;
+    if (!failed && ntile > 0) {
+      if (wait_all(o_done, (ntile - 1) & 1)) {
+        tc::fence_after();
+        have_o = true;
+      } else {
+        failed = true;
+      }
+    }
+    // epilogue: this thread's query row (loads are warp-wide, stores per row)
+    const int q = q0 + row;
+    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D;
+    const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      if (have_o) {
+        tc::tmem_ld32_sync(trow + 256u + 32u * c, ov);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) ov[k] = 0u;
+      }
+      if (q < N) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 pk;
+          pk.x = pack_bf16(__uint_as_float(ov[8 * v + 0]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
+          pk.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
+          pk.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
+          pk.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v) = pk;
+        }
+      }
+    }
+    if (q < N)
+      lse[static_cast<int64_t>(bh) * N + q] =
+          (have_o && l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+  }
+
+  if (failed) atomicOr(err_word, 1u);
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [BH][rows][D] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle, zero fill
+bool make_map(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(rows) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NST>
+cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int32_t* col_idx,
+                      int BH, int N, int G, float gbias2, void* o, float* lse,
+                      unsigned int* err_word, cudaStream_t stream) {
+  using L = FwdTcLayout<D, NST>;
+  const int nb = (N + kBlock - 1) / kBlock;
+  const float c2 = kLog2e / sqrtf(static_cast<float>(D));
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
+  fwd_tc_kernel<D, NST><<<dim3(nb, BH), kFwdTcThreads, L::kSmem, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, N, nb, G, gbias2, c2,
+      static_cast<__nv_bfloat16*>(o), lse, err_word, limit);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                          const int32_t* col_idx, const void* kg, const void* vg, int BH, int N,
+                          int d, int global_window, void* o, float* lse, unsigned int* err_word,
+                          cudaStream_t stream) {
+  const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
+  const float gbias2 = global_window > 0 ? log2f(static_cast<float>(global_window)) : 0.f;
+  CUtensorMap maps[5];
+  if (!make_map(&maps[0], qp, BH, N, d) || !make_map(&maps[1], kp, BH, N, d) ||
+      !make_map(&maps[2], vp, BH, N, d))
+    return cudaErrorInvalidValue;
+  if (G > 0) {
+    if (!make_map(&maps[3], kg, BH, G, d) || !make_map(&maps[4], vg, BH, G, d))
+      return cudaErrorInvalidValue;
+  } else {
+    maps[3] = maps[1];
+    maps[4] = maps[2];
+  }
+  if (d == 128) return launch_tc<128, 3>(maps, row_ptr, col_idx, BH, N, G, gbias2, o, lse, err_word, stream);
+  return launch_tc<64, 6>(maps, row_ptr, col_idx, BH, N, G, gbias2, o, lse, err_word, stream);
+}
+
+}  // namespace asa
