@@ -159,8 +159,12 @@ size_t asa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
  * Backward of standard ASA under the fixed mask (the mask is not differentiated):
- *   P = exp(S - LSE), D = rowsum(dO * O), dV = P^T dO, dS = P * (dO V^T - D),
- *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), all over kept tiles only.
+ *   P = exp(S - LSE), dP = dO V^T, D = rowsum(P * dP), dS = P * (dP - D),
+ *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), dV = P^T dO, all over kept tiles only.
+ * D equals rowsum(dO * O) in exact arithmetic; it is recomputed in fp32 from the kept
+ * tiles because the bf16-rounded O would cost ~4e-3 relative L2 on dQ.  `o` is
+ * validated but not read.  dS enters the dQ and dK products in fp16, so Q and K
+ * magnitudes must stay below 65504.
  * qp, kp, vp, o, dout: device bf16 [B, H, N, d]; lse: device fp32 [B, H, N] from the
  * forward; row_ptr/col_idx and col_ptr_t/row_idx_t: both CSRs of asa_build_mask;
  * dq, dk, dv: device bf16 [B, H, N, d] (fully written; no accumulation into them).

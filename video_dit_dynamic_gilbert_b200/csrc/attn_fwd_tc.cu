@@ -12,10 +12,11 @@
 //               S_{j+1} is issued before PV_j so it overlaps the softmax of tile j.
 //   warps 2..5  softmax warpgroup: thread = query row = TMEM lane.  Reads S_j,
 //               masks columns past the tile's valid rows, keeps the running max /
-//               sum in the log2 domain, writes P_j as bf16 over S_j in TMEM, and
-//               rescales O in TMEM only when the running max grows by more than
-//               2^8 (until then P is taken against the stale max; exact after the
-//               final division).  Epilogue: O / l -> bf16 rows, LSE (natural log).
+//               sum in the log2 domain, computes P_j = exp2(.) into registers while
+//               PV_{j-1} still runs, then waits for PV_{j-1}, rescales O in TMEM only
+//               when the running max grew by more than 2^8 (until then P is taken
+//               against the stale max; exact after the final division), and writes
+//               P_j as bf16 over S_j.  Epilogue: O / l -> bf16 rows, LSE (natural log).
 // TMEM: S buffers at columns [0,128) and [128,256), O at [256, 256+D).
 // Every wait is bounded: on expiry the kernel sets the device error word, drains its
 // own copies and MMAs, frees TMEM and returns.
@@ -241,30 +242,52 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       tc::fence_after();
       const TileSrc t = tile_src(j, nfine, cols, N, G);
       const float bias = t.global ? gbias2 : 0.f;
+      const bool full = t.nvalid == kBlock;
       uint32_t s[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32_sync(trow + 128u * b + 32u * c, s + 32 * c);
-      float mx = -INFINITY;
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32(trow + 128u * b + 32u * c, s + 32 * c);
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        const float x = k < t.nvalid ? fmaf(__uint_as_float(s[k]), c2, bias) : -INFINITY;
-        s[k] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int c = 0; c < 4; ++c) tc::tmem_wait_ld_dep32(s + 32 * c);
+      // row max on the raw scores (c2 > 0 keeps the order)
+      float mraw = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k) mraw = fmaxf(mraw, __uint_as_float(s[k]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k < t.nvalid) mraw = fmaxf(mraw, __uint_as_float(s[k]));
       }
+      const float mx = fmaf(mraw, c2, bias);
       const float m_new = fmaxf(m_ref, mx);
+      const bool need = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + 8.f);
+      const bool any_need = __any_sync(0xffffffffu, need) != 0;
+      const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
+      if (need) m_ref = m_new;
+      // P = exp2(s c2 + bias - m), packed to bf16 pairs
+      const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
+      uint32_t p[64];
+      float rs = 0.f;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        float a = fast_exp2(fmaf(__uint_as_float(s[2 * k]), c2, off));
+        float bb = fast_exp2(fmaf(__uint_as_float(s[2 * k + 1]), c2, off));
+        if (!full) {
+          a = 2 * k < t.nvalid ? a : 0.f;
+          bb = 2 * k + 1 < t.nvalid ? bb : 0.f;
+        }
+        rs += a + bb;
+        p[k] = pack_bf16(a, bb);
+      }
+      l = l * alpha + rs;
       if (j > 0) {
-        // PV_{j-1} done: O is stable (and the o_done phases stay in step)
+        // PV_{j-1} done: O may be rescaled, and P_j may overwrite nothing in use
         if (!wait_all(o_done, (j - 1) & 1)) {
           failed = true;
           break;
         }
         tc::fence_after();
-      }
-      const bool need = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + 8.f);
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
-        l *= alpha;
-        if (j > 0) {
+        if (any_need) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
@@ -276,19 +299,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
             tc::tmem_wait_st();
           }
         }
-        if (need) m_ref = m_new;
       }
-      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-      uint32_t p[64];
-      float rs = 0.f;
-#pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float a = fast_exp2(__uint_as_float(s[2 * k]) - mu);
-        const float bb = fast_exp2(__uint_as_float(s[2 * k + 1]) - mu);
-        rs += a + bb;
-        p[k] = pack_bf16(a, bb);
-      }
-      l += rs;
 #pragma unroll
       for (int c = 0; c < 4; ++c) tc::tmem_st16(trow + 128u * b + 16u * c, p + 16 * c);
       tc::tmem_wait_st();
