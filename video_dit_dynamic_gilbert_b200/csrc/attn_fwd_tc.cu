@@ -30,7 +30,7 @@ namespace asa {
 
 namespace {
 
-constexpr int kFwdTcThreads = 192;
+constexpr int kFwdTcThreads = 320;  // producer, MMA, 2 softmax warpgroups
 constexpr uint32_t kTmemCols = 512;
 
 template <int D, int NST>
@@ -43,10 +43,42 @@ struct FwdTcLayout {
   // barriers: q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2],
   //           o_done, drain; then the TMEM base address slot
   static constexpr uint32_t kNumBars = 1 + 3 * NST + 2 + 2 + 1 + 1;
-  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr uint32_t kRed = kBars + 8 * kNumBars;    // [2 warpgroups][128 rows] fp32
+  static constexpr uint32_t kTmemSlot = kRed + 2 * 128 * 4;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // + alignment slack
 };
+
+// exp2 on the FMA pipe: 2^x = 2^n 2^f, n = round(x) (via the 1.5*2^23 rounding
+// constant), f in [-1/2, 1/2], 2^f by a degree-3 minimax polynomial (relative error
+// 7.5e-5; coefficients from csrc/gen_exp2_poly.py).  x is clamped at -125 so that the
+// exponent add stays in the normal range.  Used for a share of the softmax
+// exponentials so that MUFU and the FMA pipe split the work.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float j = x + 12582912.f;
+  const float f = x - (j - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
+                       9.999280572e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// barrier over `nthreads` threads that also returns the AND of every thread's `v`
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return out != 0;
+}
 
 struct TileSrc {
   int row0, nvalid;
@@ -110,7 +142,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full(b), 1);
-      tc::mbar_init(p_full(b), 128);
+      tc::mbar_init(p_full(b), 256);
     }
     tc::mbar_init(o_done, 1);
     tc::mbar_init(drain, 1);
@@ -223,58 +255,80 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
+    // ------------------------------------------------------------ softmax warpgroups
+    // Two warpgroups share each row: warpgroup wg owns columns [64 wg, 64 wg + 64) of
+    // every S tile, of P and of O; the row max is combined through shared memory.
+    // tcgen05.ld/st are warp-collective and the named barriers span both warpgroups:
+    // every wait result is AND-reduced over all 256 softmax threads, so that every
+    // branch (including a timeout) is taken by all of them together.
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+    const int col0 = 64 * wg;
+    float* red = reinterpret_cast<float*>(sbase + L::kRed);
+    // bounded wait, result identical in all 256 softmax threads (barrier `id`)
+    auto wait_all = [&](uint32_t bar, uint32_t parity, int id) {
       const bool ok = tc::mbar_wait(bar, parity, wait_limit);
-      return __all_sync(0xffffffffu, ok) != 0;
+      __syncwarp();
+      return named_bar_and(id, 256, ok);
     };
     float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < ntile; ++j) {
       const int b = j & 1;
-      if (!wait_all(s_full(b), (j >> 1) & 1)) {
+      // (barrier 2 also orders this tile's exchange after the partner's last read)
+      if (!wait_all(s_full(b), (j >> 1) & 1, 2)) {
         failed = true;
         break;
       }
       tc::fence_after();
       const TileSrc t = tile_src(j, nfine, cols, N, G);
       const float bias = t.global ? gbias2 : 0.f;
-      const bool full = t.nvalid == kBlock;
-      uint32_t s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32(trow + 128u * b + 32u * c, s + 32 * c);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_wait_ld_dep32(s + 32 * c);
-      // row max on the raw scores (c2 > 0 keeps the order)
+      const int nv = t.nvalid - col0;  // valid columns in this half (may be <= 0 or >= 64)
+      const bool full = nv >= 64;
+      uint32_t s[64];
+      tc::tmem_ld32(trow + 128u * b + col0, s);
+      tc::tmem_ld32(trow + 128u * b + col0 + 32u, s + 32);
+      tc::tmem_wait_ld_dep32(s);
+      tc::tmem_wait_ld_dep32(s + 32);
+      // row max on the raw scores (c2 > 0 keeps the order), combined across halves
       float mraw = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int k = 0; k < 128; ++k) mraw = fmaxf(mraw, __uint_as_float(s[k]));
+        for (int k = 0; k < 64; ++k) mraw = fmaxf(mraw, __uint_as_float(s[k]));
       } else {
 #pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (k < t.nvalid) mraw = fmaxf(mraw, __uint_as_float(s[k]));
+        for (int k = 0; k < 64; ++k)
+          if (k < nv) mraw = fmaxf(mraw, __uint_as_float(s[k]));
       }
+      red[wg * 128 + row] = mraw;
+      named_bar_sync(1, 256);
+      mraw = fmaxf(mraw, red[(1 - wg) * 128 + row]);
       const float mx = fmaf(mraw, c2, bias);
       const float m_new = fmaxf(m_ref, mx);
       const bool need = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + 8.f);
       const bool any_need = __any_sync(0xffffffffu, need) != 0;
       const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
       if (need) m_ref = m_new;
-      // P = exp2(s c2 + bias - m), packed to bf16 pairs
+      // P = exp2(s c2 + bias - m) packed to bf16 pairs; every fourth pair on the FMA pipe
       const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
-      uint32_t p[64];
+      uint32_t p[32];
       float rs = 0.f;
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        float a = fast_exp2(fmaf(__uint_as_float(s[2 * k]), c2, off));
-        float bb = fast_exp2(fmaf(__uint_as_float(s[2 * k + 1]), c2, off));
+      for (int k = 0; k < 32; ++k) {
+        const float xa = fmaf(__uint_as_float(s[2 * k]), c2, off);
+        const float xb = fmaf(__uint_as_float(s[2 * k + 1]), c2, off);
+        float a, bb;
+        if ((k & 3) == 3) {
+          a = exp2_fma(xa);
+          bb = exp2_fma(xb);
+        } else {
+          a = fast_exp2(xa);
+          bb = fast_exp2(xb);
+        }
         if (!full) {
-          a = 2 * k < t.nvalid ? a : 0.f;
-          bb = 2 * k + 1 < t.nvalid ? bb : 0.f;
+          a = 2 * k < nv ? a : 0.f;
+          bb = 2 * k + 1 < nv ? bb : 0.f;
         }
         rs += a + bb;
         p[k] = pack_bf16(a, bb);
@@ -282,48 +336,54 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       l = l * alpha + rs;
       if (j > 0) {
         // PV_{j-1} done: O may be rescaled, and P_j may overwrite nothing in use
-        if (!wait_all(o_done, (j - 1) & 1)) {
+        if (!wait_all(o_done, (j - 1) & 1, 3)) {
           failed = true;
           break;
         }
         tc::fence_after();
         if (any_need) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
+            const uint32_t oc = trow + 256u + (D / 2) * wg + 32u * c;
             uint32_t ov[32];
-            tc::tmem_ld32_sync(trow + 256u + 32u * c, ov);
+            tc::tmem_ld32_sync(oc, ov);
 #pragma unroll
             for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-            tc::tmem_st16(trow + 256u + 32u * c, ov);
-            tc::tmem_st16(trow + 256u + 32u * c + 16u, ov + 16);
+            tc::tmem_st16(oc, ov);
+            tc::tmem_st16(oc + 16u, ov + 16);
             tc::tmem_wait_st();
           }
         }
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_st16(trow + 128u * b + 16u * c, p + 16 * c);
+      tc::tmem_st16(trow + 128u * b + 32u * wg, p);
+      tc::tmem_st16(trow + 128u * b + 32u * wg + 16u, p + 16);
       tc::tmem_wait_st();
       tc::fence_before();
       tc::mbar_arrive(p_full(b));
     }
     bool have_o = false;
     if (!failed && ntile > 0) {
-      if (wait_all(o_done, (ntile - 1) & 1)) {
+      if (wait_all(o_done, (ntile - 1) & 1, 3)) {
         tc::fence_after();
         have_o = true;
       } else {
         failed = true;
       }
     }
-    // epilogue: this thread's query row (loads are warp-wide, stores per row)
+    // row sum across the two halves
+    named_bar_sync(2, 256);
+    red[wg * 128 + row] = l;
+    named_bar_sync(1, 256);
+    const float l_row = l + red[(1 - wg) * 128 + row];
+    // epilogue: this thread's query row, columns [D/2 wg, D/2 wg + D/2)
     const int q = q0 + row;
-    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D;
-    const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D + (D / 2) * wg;
+    const float inv = (have_o && l_row > 0.f) ? 1.f / l_row : 0.f;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       uint32_t ov[32];
       if (have_o) {
-        tc::tmem_ld32_sync(trow + 256u + 32u * c, ov);
+        tc::tmem_ld32_sync(trow + 256u + (D / 2) * wg + 32u * c, ov);
       } else {
 #pragma unroll
         for (int k = 0; k < 32; ++k) ov[k] = 0u;
@@ -340,9 +400,9 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         }
       }
     }
-    if (q < N)
+    if (q < N && wg == 0)
       lse[static_cast<int64_t>(bh) * N + q] =
-          (have_o && l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+          (have_o && l_row > 0.f) ? (m_ref + __log2f(l_row)) * kLn2 : -INFINITY;
   }
 
   if (failed) atomicOr(err_word, 1u);
