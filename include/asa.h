@@ -122,6 +122,29 @@ int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* wor
                    size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
                    int32_t* col_ptr_t, int32_t* row_idx_t, void* stream);
 
+/*
+ * asa_estimate without any allocation and without a caller workspace, for callers
+ * that cannot allocate device memory (a host engine that owns all GPU memory in a
+ * fixed pool and forbids third-party allocations, or a latency-critical loop that
+ * must not risk the synchronisation cudaMalloc may cause).  The paper has no
+ * counterpart: this is a library convenience.  Same arguments, layouts and result
+ * as asa_estimate minus the workspace.
+ *   - Scratch: one file-scope device array of ASA_NOALLOC_SCRATCH_BYTES, reserved on
+ *     every device that loads the library and held until the process exits.  Shapes
+ *     needing more (4 * B*H*16*nb*(nb+1) bytes) are rejected with ASA_ERR_WORKSPACE
+ *     before anything is launched.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the array and overwrites what it reads (nothing in it needs to
+ *     start at zero).  Calls whose kernels overlap on the GPU (different streams, or
+ *     several host threads) race on the array: serialise them.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define ASA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int asa_estimate_noalloc(const void* qp, const void* kp, int B, int H, int N, int d, int block,
+                         int samples, float* p_imp, void* stream);
+
 /* Steps 1 + 2.1 in one call (P_imp stays in the workspace). Arguments as above. */
 int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d, int block,
                       int samples, float tau, void* workspace, size_t ws_bytes, int32_t* row_ptr,

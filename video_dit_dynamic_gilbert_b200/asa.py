@@ -35,6 +35,7 @@ _SIGNATURES = {
     "asa_unpermute": ([_vp, _vp] + [_c_int] * 6 + [_vp], _c_int),
     "asa_estimate_mask_workspace_size": ([_c_int] * 3, _c_size),
     "asa_estimate": ([_vp, _vp] + [_c_int] * 6 + [_vp, _c_size, _vp, _vp], _c_int),
+    "asa_estimate_noalloc": ([_vp, _vp] + [_c_int] * 6 + [_vp, _vp], _c_int),
     "asa_build_mask": ([_vp, _c_int, _c_int, _c_int, _c_float, _vp, _c_size] + [_vp] * 6, _c_int),
     "asa_estimate_mask": ([_vp, _vp] + [_c_int] * 6 + [_c_float, _vp, _c_size] + [_vp] * 6, _c_int),
     "asa_global_pool": ([_vp, _vp] + [_c_int] * 5 + [_vp], _c_int),
@@ -185,6 +186,21 @@ def asa_estimate(qp: torch.Tensor, kp: torch.Tensor, workspace=None, out=None, s
         out = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qp.device)
     _check(lib().asa_estimate(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, _ptr(workspace),
                               workspace.numel(), _ptr(out), _stream(stream)))
+    return out
+
+
+def asa_estimate_noalloc(qp: torch.Tensor, kp: torch.Tensor, out=None, stream=None):
+    """asa_estimate with its scratch in the library's fixed device array (no workspace,
+    no allocation in the library; for callers that cannot allocate device memory).
+    Calls that overlap on the GPU share that array and race: serialise them."""
+    _bf16_cuda("qp", qp)
+    _bf16_cuda("kp", kp)
+    B, H, N, d = qp.shape
+    nb = nblocks(N)
+    if out is None:
+        out = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qp.device)
+    _check(lib().asa_estimate_noalloc(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, _ptr(out),
+                                      _stream(stream)))
     return out
 
 

@@ -173,6 +173,18 @@ int check_block(int block, int samples) {
 
 __device__ unsigned int g_device_error = 0;
 
+namespace asa {
+int record_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+}  // namespace asa
+
 namespace {
 // Device address of g_device_error for the current device (kernels set bits in it
 // when a bounded wait expires).

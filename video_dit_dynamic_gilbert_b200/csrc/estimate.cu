@@ -11,6 +11,9 @@
 //     max logit G[bh, J, r]; at the end lse2[bh, r] = m + log2(l).
 //   est_pool:   P_imp[bh, I, J] = max_{r in I} exp2(G[bh, J, r] - lse2[bh, r]).
 // G (16 * nb floats per key block and head) lives in the caller's workspace.
+#include <mutex>
+
+#include "../../include/asa.h"
 #include "common.cuh"
 #include "internal.h"
 
@@ -234,3 +237,84 @@ cudaError_t launch_estimate(const void* qp, const void* kp, int BH, int N, int d
 }
 
 }  // namespace asa
+
+// ---------------------------------------------------------------------------------
+// Allocation-free variant of asa_estimate.
+//
+// Some callers cannot allocate device memory at all: code embedded in a host
+// application or inference engine that owns every byte of the GPU through its own
+// fixed, pre-reserved pool and forbids third-party allocations, or a latency-critical
+// loop that must not risk the device-wide synchronisation cudaMalloc / cudaFree can
+// cause.  For them the estimator's scratch (per sample row, the max logit of every key
+// block, and the row's log2-sum-exp) lives in one file-scope device array of fixed
+// size, reserved when the library is loaded on a device and held until the process
+// exits.  The caller still passes the inputs and the P_imp output.
+namespace {
+
+constexpr size_t kNoallocScratchFloats = ASA_NOALLOC_SCRATCH_BYTES / sizeof(float);
+static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[64] = {nullptr};
+
+// Device address of the scratch array on the current device, looked up once per
+// device (the host-side name of the array is not a device address).
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess)
+    return asa::record_error(ASA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return asa::record_error(ASA_ERR_UNSUPPORTED, "device %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return asa::record_error(ASA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s",
+                               cudaGetErrorString(e));
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return ASA_OK;
+}
+
+}  // namespace
+
+extern "C" int asa_estimate_noalloc(const void* qp, const void* kp, int B, int H, int N, int d,
+                                    int block, int samples, float* p_imp, void* stream) {
+  if (B < 1 || H < 1 || N < 1)
+    return asa::record_error(ASA_ERR_INVALID_ARG, "B=%d, H=%d, N=%d must be >= 1", B, H, N);
+  if (static_cast<int64_t>(B) * H > 65535 || N > ASA_MAX_TOKENS)
+    return asa::record_error(ASA_ERR_UNSUPPORTED, "B*H=%lld or N=%d too large",
+                             static_cast<long long>(B) * H, N);
+  if (d != 64 && d != 128)
+    return asa::record_error(ASA_ERR_UNSUPPORTED, "head dim d=%d not in {64,128}", d);
+  if (block != ASA_BLOCK || samples != ASA_SAMPLES)
+    return asa::record_error(ASA_ERR_UNSUPPORTED, "block=%d, samples=%d (only 128, 16)", block,
+                             samples);
+  if (qp == nullptr || kp == nullptr || p_imp == nullptr)
+    return asa::record_error(ASA_ERR_INVALID_ARG, "qp, kp and p_imp must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(qp) & 15u) || (reinterpret_cast<uintptr_t>(kp) & 15u) ||
+      (reinterpret_cast<uintptr_t>(p_imp) & 3u))
+    return asa::record_error(ASA_ERR_INVALID_ARG, "qp/kp need 16-byte, p_imp 4-byte alignment");
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  const size_t need = asa::est_scratch_floats(B * H, nb);
+  if (need > kNoallocScratchFloats)
+    return asa::record_error(ASA_ERR_WORKSPACE,
+                             "shape needs %zu bytes of scratch, above the fixed %zu bytes of "
+                             "asa_estimate_noalloc",
+                             need * sizeof(float), static_cast<size_t>(ASA_NOALLOC_SCRATCH_BYTES));
+  float* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != ASA_OK) return rc;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  float* G = scratch;
+  float* lse2 = scratch + static_cast<size_t>(B) * H * nb * asa::kSamplesHost * nb;
+  cudaError_t e = asa::launch_estimate(qp, kp, B * H, N, d, G, lse2, p_imp, sms,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return asa::record_error(ASA_ERR_CUDA, "estimate launch: %s", cudaGetErrorString(e));
+  return ASA_OK;
+}

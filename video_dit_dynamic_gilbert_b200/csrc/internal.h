@@ -11,6 +11,9 @@ constexpr int kSamplesHost = 16;  // k: sampled tokens per block
 
 bool gilbert_order_host(int T, int Hg, int W, int32_t* out);
 
+// Records the calling thread's error message for asa_last_error_string(); returns code.
+int record_error(int code, const char* fmt, ...);
+
 cudaError_t launch_permute(const void* const* src, void* const* dst, int ntensors, bool to_permuted,
                            const int32_t* perm_dev, int B, int N, int H, int d, int num_sms,
                            cudaStream_t stream);
