@@ -63,6 +63,16 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).  The forward is issue-
+// bound in the softmax, where a MUFU exp2 costs one instruction and exp2_fma nine.
+constexpr int kPolyEvery = 0;
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -285,22 +295,26 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       const TileSrc t = tile_src(j, nfine, cols, N, G);
       const float bias = t.global ? gbias2 : 0.f;
       const int nv = t.nvalid - col0;  // valid columns in this half (may be <= 0 or >= 64)
-      const bool full = nv >= 64;
       uint32_t s[64];
       tc::tmem_ld32(trow + 128u * b + col0, s);
       tc::tmem_ld32(trow + 128u * b + col0 + 32u, s + 32);
       tc::tmem_wait_ld_dep32(s);
       tc::tmem_wait_ld_dep32(s + 32);
-      // row max on the raw scores (c2 > 0 keeps the order), combined across halves
-      float mraw = -INFINITY;
-      if (full) {
-#pragma unroll
-        for (int k = 0; k < 64; ++k) mraw = fmaxf(mraw, __uint_as_float(s[k]));
-      } else {
+      // full tiles skip every per-column validity test
+      if (nv < 64) {
 #pragma unroll
         for (int k = 0; k < 64; ++k)
-          if (k < nv) mraw = fmaxf(mraw, __uint_as_float(s[k]));
+          if (k >= nv) s[k] = __float_as_uint(-INFINITY);
       }
+      // row max on the raw scores (c2 > 0 keeps the order), combined across halves
+      float m0 = max3f(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
+      float m1 = max3f(__uint_as_float(s[3]), __uint_as_float(s[4]), __uint_as_float(s[5]));
+#pragma unroll
+      for (int k = 6; k < 62; k += 4) {
+        m0 = max3f(m0, __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
+        m1 = max3f(m1, __uint_as_float(s[k + 2]), __uint_as_float(s[k + 3]));
+      }
+      float mraw = max3f(m0, m1, fmaxf(__uint_as_float(s[62]), __uint_as_float(s[63])));
       red[wg * 128 + row] = mraw;
       named_bar_sync(1, 256);
       mraw = fmaxf(mraw, red[(1 - wg) * 128 + row]);
@@ -310,29 +324,27 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       const bool any_need = __any_sync(0xffffffffu, need) != 0;
       const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
       if (need) m_ref = m_new;
-      // P = exp2(s c2 + bias - m) packed to bf16 pairs; every fourth pair on the FMA pipe
+      // P = exp2(s c2 + bias - m) packed to bf16 pairs (masked columns give exp2(-inf) = 0)
       const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
       uint32_t p[32];
-      float rs = 0.f;
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float xa = fmaf(__uint_as_float(s[2 * k]), c2, off);
         const float xb = fmaf(__uint_as_float(s[2 * k + 1]), c2, off);
         float a, bb;
-        if ((k & 3) == 3) {
+        if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == 0) {
           a = exp2_fma(xa);
           bb = exp2_fma(xb);
         } else {
           a = fast_exp2(xa);
           bb = fast_exp2(xb);
         }
-        if (!full) {
-          a = 2 * k < nv ? a : 0.f;
-          bb = 2 * k + 1 < nv ? bb : 0.f;
-        }
-        rs += a + bb;
+        rs0 += a;
+        rs1 += bb;
         p[k] = pack_bf16(a, bb);
       }
+      const float rs = rs0 + rs1;
       l = l * alpha + rs;
       if (j > 0) {
         // PV_{j-1} done: O may be rescaled, and P_j may overwrite nothing in use
