@@ -1,25 +1,27 @@
 // Block-sparse attention forward on tcgen05 tensor cores (Video-BLADE, "Step 2.2:
 // Computation": standard ASA over the kept tiles of M, and ASA_G with global tokens).
 //
-// One CTA per (b, h, query block I of 128 rows), 6 warps, warp-specialised:
+// One CTA per (b, h, query block I of 128 rows), 10 warps, warp-specialised:
 //   warp 0      TMA producer: Q once, then for every kept key block J (the CSR row
 //               of I) its 128-row K and V tiles into an NST-stage ring; for ASA_G
-//               then the ceil(N/n) global tokens in 128-row tiles.  Tiles past N
+//               then the ceil(N/n) global tokens in 128-row tiles.  Rows past N
 //               (ragged last block) are zero-filled by TMA.
 //   warp 1      TMEM owner and MMA issuer (one thread):
-//                 S_j = Q K_j^T   (SS MMA, M=128 N=128, into TMEM S buffer j%2)
-//                 O  += P_j V_j   (TS MMA: P read from TMEM, V from shared memory)
-//               S_{j+1} is issued before PV_j so it overlaps the softmax of tile j.
-//   warps 2..5  softmax warpgroup: thread = query row = TMEM lane.  Reads S_j,
-//               masks columns past the tile's valid rows, keeps the running max /
-//               sum in the log2 domain, computes P_j = exp2(.) into registers while
-//               PV_{j-1} still runs, then waits for PV_{j-1}, rescales O in TMEM only
-//               when the running max grew by more than 2^8 (until then P is taken
-//               against the stale max; exact after the final division), and writes
-//               P_j as bf16 over S_j.  Epilogue: O / l -> bf16 rows, LSE (natural log).
-// TMEM: S buffers at columns [0,128) and [128,256), O at [256, 256+D).
-// Every wait is bounded: on expiry the kernel sets the device error word, drains its
-// own copies and MMAs, frees TMEM and returns.
+//                 S_j = Q K_j^T   (SS MMA, M=128 N=128) into TMEM S buffer j%2,
+//                 O_{j%2} += P_j V_j   (TS MMA: P read from TMEM, V from shared memory).
+//   warps 2..9  two softmax warpgroups.  Warpgroup w takes the tiles j = w, w+2, ...:
+//               an independent online softmax (running max / sum in the log2 domain)
+//               with its own S buffer and its own O accumulator, so that one
+//               warpgroup's loads, reductions and stores overlap the other's exp2 work
+//               and the tensor pipe always has a tile to run.  Thread = query row =
+//               TMEM lane.  P_j is written as bf16 over S_j; O is rescaled in TMEM only
+//               when the running max grows by more than 2^8 (until then P is taken
+//               against the stale max; exact after the final division).  Epilogue:
+//               the two partial results are merged (max, scaled sums) and O / l is
+//               written as bf16 rows with the natural-log LSE.
+// TMEM: S buffers at columns [0,128) and [128,256), O_0 at [256,256+D), O_1 at
+// [384,384+D).  Every wait is bounded: on expiry the kernel sets the device error word,
+// drains its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -41,10 +43,9 @@ struct FwdTcLayout {
   static constexpr uint32_t kV = kK + NST * kTile;
   static constexpr uint32_t kBars = kV + NST * kTile;
   // barriers: q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2],
-  //           o_done, drain; then the TMEM base address slot
-  static constexpr uint32_t kNumBars = 1 + 3 * NST + 2 + 2 + 1 + 1;
-  static constexpr uint32_t kRed = kBars + 8 * kNumBars;    // [2 warpgroups][128 rows] fp32
-  static constexpr uint32_t kTmemSlot = kRed + 2 * 128 * 4;
+  //           o_done[2], drain; then the TMEM base address slot
+  static constexpr uint32_t kNumBars = 1 + 3 * NST + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // + alignment slack
 };
@@ -69,25 +70,11 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).  The forward is issue-
-// bound in the softmax, where a MUFU exp2 costs one instruction and exp2_fma nine.
+// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).
 constexpr int kPolyEvery = 0;
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// barrier over `nthreads` threads that also returns the AND of every thread's `v`
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}\n"
-      : "=r"(out)
-      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
-      : "memory");
-  return out != 0;
 }
 
 struct TileSrc {
@@ -139,8 +126,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NST + s); };
   auto s_full = [&](int b) { return bar0 + 8u * (1 + 3 * NST + b); };
   auto p_full = [&](int b) { return bar0 + 8u * (3 + 3 * NST + b); };
-  const uint32_t o_done = bar0 + 8u * (5 + 3 * NST);
-  const uint32_t drain = bar0 + 8u * (6 + 3 * NST);
+  auto o_done = [&](int b) { return bar0 + 8u * (5 + 3 * NST + b); };
+  const uint32_t drain = bar0 + 8u * (7 + 3 * NST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kTmemSlot);
 
   if (threadIdx.x == 0) {
@@ -152,9 +139,9 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full(b), 1);
-      tc::mbar_init(p_full(b), 256);
+      tc::mbar_init(p_full(b), 128);
+      tc::mbar_init(o_done(b), 1);
     }
-    tc::mbar_init(o_done, 1);
     tc::mbar_init(drain, 1);
     tc::fence_barrier_init();
   }
@@ -214,11 +201,10 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idPV = tc::idesc_bf16(128, D, false, true);
-      const uint32_t tO = tmem + 256u;
+      // S_j = Q K_j^T into S buffer j % 2
       auto issue_s = [&](int j) {
-        const int st = j % NST;
         const uint32_t dS = tmem + 128u * (j & 1);
-        const uint32_t kb = base + L::kK + st * L::kTile;
+        const uint32_t kb = base + L::kK + (j % NST) * L::kTile;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
@@ -228,34 +214,36 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       };
       bool ok = tc::mbar_wait(q_full(), 0, wait_limit);
       int issued_any = 0;
-      if (ok && ntile > 0) {
-        ok = tc::mbar_wait(k_full(0), 0, wait_limit);
-        if (ok) {
-          tc::fence_after();
-          issue_s(0);
-          tc::umma_commit(s_full(0));
-          issued_any = 1;
-        }
+      // the first tile of each stream
+      for (int j = 0; ok && j < 2 && j < ntile; ++j) {
+        if (!(ok = tc::mbar_wait(k_full(j % NST), (j / NST) & 1, wait_limit))) break;
+        tc::fence_after();
+        issue_s(j);
+        tc::umma_commit(s_full(j & 1));
+        issued_any = 1;
       }
       for (int j = 0; ok && j < ntile; ++j) {
-        if (j + 1 < ntile) {
-          const int st1 = (j + 1) % NST;
-          if (!(ok = tc::mbar_wait(k_full(st1), ((j + 1) / NST) & 1, wait_limit))) break;
-          tc::fence_after();
-          issue_s(j + 1);
-          tc::umma_commit(s_full((j + 1) & 1));
-        }
-        if (!(ok = tc::mbar_wait(p_full(j & 1), (j >> 1) & 1, wait_limit))) break;
+        const int b = j & 1;
+        if (!(ok = tc::mbar_wait(p_full(b), (j >> 1) & 1, wait_limit))) break;
         if (!(ok = tc::mbar_wait(v_full(j % NST), (j / NST) & 1, wait_limit))) break;
         tc::fence_after();
-        const uint32_t tP = tmem + 128u * (j & 1);
+        // O_b += P_j V_j; the first tile of a stream initialises its O
+        const uint32_t tP = tmem + 128u * b;
+        const uint32_t tO = tmem + 256u + 128u * b;
         const uint32_t vb = base + L::kV + (j % NST) * L::kTile;
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
           tc::umma_ts(tO, tP + 8u * ks, tc::sdesc_sw128(vb + ks * 2048u, 16384, 1024), idPV,
-                      (j > 0 || ks > 0) ? 1u : 0u);
+                      (j >= 2 || ks > 0) ? 1u : 0u);
         tc::umma_commit(kv_empty(j % NST));
-        tc::umma_commit(o_done);
+        tc::umma_commit(o_done(b));
+        // the stream's next S goes into the buffer P_j just left (in issue order)
+        if (j + 2 < ntile) {
+          if (!(ok = tc::mbar_wait(k_full((j + 2) % NST), ((j + 2) / NST) & 1, wait_limit))) break;
+          tc::fence_after();
+          issue_s(j + 2);
+          tc::umma_commit(s_full(b));
+        }
       }
       failed = !ok;
       if (issued_any) {
@@ -266,58 +254,48 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    // Two warpgroups share each row: warpgroup wg owns columns [64 wg, 64 wg + 64) of
-    // every S tile, of P and of O; the row max is combined through shared memory.
-    // tcgen05.ld/st are warp-collective and the named barriers span both warpgroups:
-    // every wait result is AND-reduced over all 256 softmax threads, so that every
-    // branch (including a timeout) is taken by all of them together.
-    const int wg = (warp - 2) >> 2;
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
+    // (wait results are AND-reduced over the warp).
+    const int w = (warp - 2) >> 2;  // stream: tiles w, w + 2, ...
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const int col0 = 64 * wg;
-    float* red = reinterpret_cast<float*>(sbase + L::kRed);
-    // bounded wait, result identical in all 256 softmax threads (barrier `id`)
-    auto wait_all = [&](uint32_t bar, uint32_t parity, int id) {
+    const uint32_t tS = trow + 128u * w;
+    const uint32_t tO = trow + 256u + 128u * w;
+    auto wait_warp = [&](uint32_t bar, uint32_t parity) {
       const bool ok = tc::mbar_wait(bar, parity, wait_limit);
-      __syncwarp();
-      return named_bar_and(id, 256, ok);
+      return __all_sync(0xffffffffu, ok) != 0;
     };
     float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < ntile; ++j) {
-      const int b = j & 1;
-      // (barrier 2 also orders this tile's exchange after the partner's last read)
-      if (!wait_all(s_full(b), (j >> 1) & 1, 2)) {
+    int it = 0;  // tiles of this stream done
+    for (int j = w; j < ntile; j += 2, ++it) {
+      if (!wait_warp(s_full(w), it & 1)) {
         failed = true;
         break;
       }
       tc::fence_after();
       const TileSrc t = tile_src(j, nfine, cols, N, G);
       const float bias = t.global ? gbias2 : 0.f;
-      const int nv = t.nvalid - col0;  // valid columns in this half (may be <= 0 or >= 64)
-      uint32_t s[64];
-      tc::tmem_ld32(trow + 128u * b + col0, s);
-      tc::tmem_ld32(trow + 128u * b + col0 + 32u, s + 32);
-      tc::tmem_wait_ld_dep32(s);
-      tc::tmem_wait_ld_dep32(s + 32);
-      // full tiles skip every per-column validity test
-      if (nv < 64) {
+      uint32_t s[128];
 #pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (k >= nv) s[k] = __float_as_uint(-INFINITY);
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS + 32u * c, s + 32 * c);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_wait_ld_dep32(s + 32 * c);
+      // full tiles skip every per-column validity test
+      if (t.nvalid < kBlock) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k >= t.nvalid) s[k] = __float_as_uint(-INFINITY);
       }
-      // row max on the raw scores (c2 > 0 keeps the order), combined across halves
+      // row max on the raw scores (c2 > 0 keeps the order)
       float m0 = max3f(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
       float m1 = max3f(__uint_as_float(s[3]), __uint_as_float(s[4]), __uint_as_float(s[5]));
 #pragma unroll
-      for (int k = 6; k < 62; k += 4) {
+      for (int k = 6; k < 126; k += 4) {
         m0 = max3f(m0, __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
         m1 = max3f(m1, __uint_as_float(s[k + 2]), __uint_as_float(s[k + 3]));
       }
-      float mraw = max3f(m0, m1, fmaxf(__uint_as_float(s[62]), __uint_as_float(s[63])));
-      red[wg * 128 + row] = mraw;
-      named_bar_sync(1, 256);
-      mraw = fmaxf(mraw, red[(1 - wg) * 128 + row]);
+      const float mraw = max3f(m0, m1, fmaxf(__uint_as_float(s[126]), __uint_as_float(s[127])));
       const float mx = fmaf(mraw, c2, bias);
       const float m_new = fmaxf(m_ref, mx);
       const bool need = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + 8.f);
@@ -326,10 +304,10 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       if (need) m_ref = m_new;
       // P = exp2(s c2 + bias - m) packed to bf16 pairs (masked columns give exp2(-inf) = 0)
       const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
-      uint32_t p[32];
+      uint32_t p[64];
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
+      for (int k = 0; k < 64; ++k) {
         const float xa = fmaf(__uint_as_float(s[2 * k]), c2, off);
         const float xb = fmaf(__uint_as_float(s[2 * k + 1]), c2, off);
         float a, bb;
@@ -344,77 +322,103 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         rs1 += bb;
         p[k] = pack_bf16(a, bb);
       }
-      const float rs = rs0 + rs1;
-      l = l * alpha + rs;
-      if (j > 0) {
-        // PV_{j-1} done: O may be rescaled, and P_j may overwrite nothing in use
-        if (!wait_all(o_done, (j - 1) & 1, 3)) {
+      l = l * alpha + (rs0 + rs1);
+      if (it > 0) {
+        // this stream's previous PV is done: O may be rescaled
+        if (!wait_warp(o_done(w), (it - 1) & 1)) {
           failed = true;
           break;
         }
         tc::fence_after();
         if (any_need) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            const uint32_t oc = trow + 256u + (D / 2) * wg + 32u * c;
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
-            tc::tmem_ld32_sync(oc, ov);
+            tc::tmem_ld32_sync(tO + 32u * c, ov);
 #pragma unroll
             for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-            tc::tmem_st16(oc, ov);
-            tc::tmem_st16(oc + 16u, ov + 16);
+            tc::tmem_st16(tO + 32u * c, ov);
+            tc::tmem_st16(tO + 32u * c + 16u, ov + 16);
             tc::tmem_wait_st();
           }
         }
       }
-      tc::tmem_st16(trow + 128u * b + 32u * wg, p);
-      tc::tmem_st16(trow + 128u * b + 32u * wg + 16u, p + 16);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_st16(tS + 16u * c, p + 16 * c);
       tc::tmem_wait_st();
       tc::fence_before();
-      tc::mbar_arrive(p_full(b));
+      tc::mbar_arrive(p_full(w));
     }
+    // this stream's last PV
+    const bool had = !failed && it > 0;
     bool have_o = false;
-    if (!failed && ntile > 0) {
-      if (wait_all(o_done, (ntile - 1) & 1, 3)) {
+    if (had) {
+      if (wait_warp(o_done(w), (it - 1) & 1)) {
         tc::fence_after();
         have_o = true;
       } else {
         failed = true;
       }
     }
-    // row sum across the two halves
-    named_bar_sync(2, 256);
-    red[wg * 128 + row] = l;
+    // merge the two streams: (m, l) through shared memory, over Q's bytes (every MMA
+    // that reads Q is complete once both warpgroups hold their last PV)
+    float* red = reinterpret_cast<float*>(sbase + L::kQ);  // [2][2][128]: m, l per stream
     named_bar_sync(1, 256);
-    const float l_row = l + red[(1 - wg) * 128 + row];
-    // epilogue: this thread's query row, columns [D/2 wg, D/2 wg + D/2)
+    red[(2 * w) * 128 + row] = have_o ? m_ref : -INFINITY;
+    red[(2 * w + 1) * 128 + row] = have_o ? l : 0.f;
+    red[(4 + w) * 128 + row] = have_o ? 1.f : 0.f;
+    named_bar_sync(1, 256);
+    const float m_0 = red[0 * 128 + row], l_0 = red[1 * 128 + row];
+    const float m_1 = red[2 * 128 + row], l_1 = red[3 * 128 + row];
+    const bool has_0 = red[4 * 128 + row] != 0.f, has_1 = red[5 * 128 + row] != 0.f;
+    const float m = fmaxf(m_0, m_1);
+    const float s_0 = has_0 ? fast_exp2(m_0 - m) : 0.f;
+    const float s_1 = has_1 ? fast_exp2(m_1 - m) : 0.f;
+    const float l_row = l_0 * s_0 + l_1 * s_1;
+    const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+    // warpgroup w writes columns [D/2 w, D/2 w + D/2) of its rows
     const int q = q0 + row;
-    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D + (D / 2) * wg;
-    const float inv = (have_o && l_row > 0.f) ? 1.f / l_row : 0.f;
+    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D + (D / 2) * w;
+    const bool h0 = __all_sync(0xffffffffu, has_0) != 0 || __any_sync(0xffffffffu, has_0) != 0;
+    const bool h1 = __any_sync(0xffffffffu, has_1) != 0;
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      uint32_t ov[32];
-      if (have_o) {
-        tc::tmem_ld32_sync(trow + 256u + (D / 2) * wg + 32u * c, ov);
+      uint32_t a0[32], a1[32];
+      const uint32_t col = (D / 2) * w + 32u * c;
+      if (h0) {
+        tc::tmem_ld32_sync(trow + 256u + col, a0);
       } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) ov[k] = 0u;
+        for (int k = 0; k < 32; ++k) a0[k] = 0u;
       }
+      if (h1) {
+        tc::tmem_ld32_sync(trow + 384u + col, a1);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a1[k] = 0u;
+      }
+      const float f0 = s_0 * inv, f1 = s_1 * inv;
       if (q < N) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float o0 = has_0 ? __uint_as_float(a0[8 * v + e]) * f0 : 0.f;
+            const float o1 = has_1 ? __uint_as_float(a1[8 * v + e]) * f1 : 0.f;
+            x[e] = o0 + o1;
+          }
           uint4 pk;
-          pk.x = pack_bf16(__uint_as_float(ov[8 * v + 0]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
-          pk.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
-          pk.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
-          pk.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
+          pk.x = pack_bf16(x[0], x[1]);
+          pk.y = pack_bf16(x[2], x[3]);
+          pk.z = pack_bf16(x[4], x[5]);
+          pk.w = pack_bf16(x[6], x[7]);
           *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v) = pk;
         }
       }
     }
-    if (q < N && wg == 0)
-      lse[static_cast<int64_t>(bh) * N + q] =
-          (have_o && l_row > 0.f) ? (m_ref + __log2f(l_row)) * kLn2 : -INFINITY;
+    if (q < N && w == 0)
+      lse[static_cast<int64_t>(bh) * N + q] = l_row > 0.f ? (m + __log2f(l_row)) * kLn2 : -INFINITY;
   }
 
   if (failed) atomicOr(err_word, 1u);
