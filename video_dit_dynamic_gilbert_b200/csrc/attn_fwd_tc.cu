@@ -42,9 +42,9 @@ struct FwdTcLayout {
   static constexpr uint32_t kK = kQ + kTile;
   static constexpr uint32_t kV = kK + NST * kTile;
   static constexpr uint32_t kBars = kV + NST * kTile;
-  // barriers: q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2],
-  //           o_done[2], drain; then the TMEM base address slot
-  static constexpr uint32_t kNumBars = 1 + 3 * NST + 2 + 2 + 2 + 1;
+  // barriers: q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[2],
+  //           p_full[2], o_done[2], drain; then the TMEM base address slot
+  static constexpr uint32_t kNumBars = 1 + 4 * NST + 2 + 2 + 2 + 1;
   static constexpr uint32_t kTmemSlot = kBars + 8 * kNumBars;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // + alignment slack
@@ -70,8 +70,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).
-constexpr int kPolyEvery = 0;
+// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).  A single softmax warp
+// reaches only ~2.8 of MUFU's 4 exp2/clk per sub-partition; the FMA pipe has room.
+constexpr int kPolyEvery = 4;
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -123,11 +124,12 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   auto q_full = [&]() { return bar0; };
   auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto v_full = [&](int s) { return bar0 + 8u * (1 + NST + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NST + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (1 + 3 * NST + b); };
-  auto p_full = [&](int b) { return bar0 + 8u * (3 + 3 * NST + b); };
-  auto o_done = [&](int b) { return bar0 + 8u * (5 + 3 * NST + b); };
-  const uint32_t drain = bar0 + 8u * (7 + 3 * NST);
+  auto k_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NST + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (1 + 3 * NST + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (1 + 4 * NST + b); };
+  auto p_full = [&](int b) { return bar0 + 8u * (3 + 4 * NST + b); };
+  auto o_done = [&](int b) { return bar0 + 8u * (5 + 4 * NST + b); };
+  const uint32_t drain = bar0 + 8u * (7 + 4 * NST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kTmemSlot);
 
   if (threadIdx.x == 0) {
@@ -135,7 +137,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     for (int s = 0; s < NST; ++s) {
       tc::mbar_init(k_full(s), 1);
       tc::mbar_init(v_full(s), 1);
-      tc::mbar_init(kv_empty(s), 1);
+      tc::mbar_init(k_empty(s), 1);
+      tc::mbar_init(v_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full(b), 1);
@@ -156,44 +159,44 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   bool failed = false;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tc::tma_prefetch(&tmQ);
-      tc::tma_prefetch(&tmK);
-      tc::tma_prefetch(&tmV);
-      tc::mbar_expect_tx(q_full(), L::kTile);
+    // ------------------------------------------------------------ TMA producers
+    // lane 0 streams Q and the K tiles, lane 1 the V tiles: a K stage is released as
+    // soon as its S MMA completes, a V stage only after its PV MMA.
+    if (lane < 2) {
+      const bool isK = lane == 0;
+      if (isK) {
+        tc::tma_prefetch(&tmQ);
+        tc::tma_prefetch(&tmK);
+        tc::mbar_expect_tx(q_full(), L::kTile);
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h)
-        tc::tma_load_3d(base + L::kQ + h * 16384u, &tmQ, 64 * h, q0, bh, q_full());
+        for (int h = 0; h < D / 64; ++h)
+          tc::tma_load_3d(base + L::kQ + h * 16384u, &tmQ, 64 * h, q0, bh, q_full());
+      } else {
+        tc::tma_prefetch(&tmV);
+      }
+      const uint32_t ring = base + (isK ? L::kK : L::kV);
       int issued = 0;
       for (int j = 0; j < ntile; ++j) {
         const int st = j % NST, n = j / NST;
-        if (n > 0 && !tc::mbar_wait(kv_empty(st), (n - 1) & 1, wait_limit)) {
+        if (n > 0 && !tc::mbar_wait(isK ? k_empty(st) : v_empty(st), (n - 1) & 1, wait_limit)) {
           failed = true;
           break;
         }
         const TileSrc t = tile_src(j, nfine, cols, N, G);
-        const CUtensorMap* mk = t.global ? &tmKg : &tmK;
-        const CUtensorMap* mv = t.global ? &tmVg : &tmV;
-        tc::mbar_expect_tx(k_full(st), L::kTile);
+        const CUtensorMap* m = t.global ? (isK ? &tmKg : &tmVg) : (isK ? &tmK : &tmV);
+        const uint32_t full = isK ? k_full(st) : v_full(st);
+        tc::mbar_expect_tx(full, L::kTile);
 #pragma unroll
         for (int h = 0; h < D / 64; ++h)
-          tc::tma_load_3d(base + L::kK + st * L::kTile + h * 16384u, mk, 64 * h, t.row0, bh,
-                          k_full(st));
-        tc::mbar_expect_tx(v_full(st), L::kTile);
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tc::tma_load_3d(base + L::kV + st * L::kTile + h * 16384u, mv, 64 * h, t.row0, bh,
-                          v_full(st));
+          tc::tma_load_3d(ring + st * L::kTile + h * 16384u, m, 64 * h, t.row0, bh, full);
         issued = j + 1;
       }
       // drain: every issued copy has landed, and the MMAs have released the last
       // stages (their commits arrive before the CTA exits)
-      tc::mbar_wait(q_full(), 0, wait_limit);
+      if (isK) tc::mbar_wait(q_full(), 0, wait_limit);
       for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j) {
-        tc::mbar_wait(k_full(j % NST), (j / NST) & 1, wait_limit);
-        tc::mbar_wait(v_full(j % NST), (j / NST) & 1, wait_limit);
-        tc::mbar_wait(kv_empty(j % NST), (j / NST) & 1, wait_limit);
+        tc::mbar_wait(isK ? k_full(j % NST) : v_full(j % NST), (j / NST) & 1, wait_limit);
+        tc::mbar_wait(isK ? k_empty(j % NST) : v_empty(j % NST), (j / NST) & 1, wait_limit);
       }
     }
   } else if (warp == 1) {
@@ -220,12 +223,17 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         tc::fence_after();
         issue_s(j);
         tc::umma_commit(s_full(j & 1));
+        tc::umma_commit(k_empty(j % NST));
         issued_any = 1;
       }
       for (int j = 0; ok && j < ntile; ++j) {
         const int b = j & 1;
-        if (!(ok = tc::mbar_wait(p_full(b), (j >> 1) & 1, wait_limit))) break;
+        // operands first, P last: once P_j lands, PV_j and S_{j+2} issue at once
         if (!(ok = tc::mbar_wait(v_full(j % NST), (j / NST) & 1, wait_limit))) break;
+        if (j + 2 < ntile &&
+            !(ok = tc::mbar_wait(k_full((j + 2) % NST), ((j + 2) / NST) & 1, wait_limit)))
+          break;
+        if (!(ok = tc::mbar_wait(p_full(b), (j >> 1) & 1, wait_limit))) break;
         tc::fence_after();
         // O_b += P_j V_j; the first tile of a stream initialises its O
         const uint32_t tP = tmem + 128u * b;
@@ -235,14 +243,13 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         for (int ks = 0; ks < kBlock / 16; ++ks)
           tc::umma_ts(tO, tP + 8u * ks, tc::sdesc_sw128(vb + ks * 2048u, 16384, 1024), idPV,
                       (j >= 2 || ks > 0) ? 1u : 0u);
-        tc::umma_commit(kv_empty(j % NST));
+        tc::umma_commit(v_empty(j % NST));
         tc::umma_commit(o_done(b));
         // the stream's next S goes into the buffer P_j just left (in issue order)
         if (j + 2 < ntile) {
-          if (!(ok = tc::mbar_wait(k_full((j + 2) % NST), ((j + 2) / NST) & 1, wait_limit))) break;
-          tc::fence_after();
           issue_s(j + 2);
           tc::umma_commit(s_full(b));
+          tc::umma_commit(k_empty((j + 2) % NST));
         }
       }
       failed = !ok;
