@@ -1,7 +1,7 @@
 // Block-sparse attention forward on tcgen05 tensor cores (Video-BLADE, "Step 2.2:
 // Computation": standard ASA over the kept tiles of M, and ASA_G with global tokens).
 //
-// One CTA per (b, h, query block I of 128 rows), 10 warps, warp-specialised:
+// One CTA per (b, h, query block I of 128 rows), 12 warps, warp-specialised:
 //   warp 0      TMA producer: Q once, then for every kept key block J (the CSR row
 //               of I) its 128-row K and V tiles into an NST-stage ring; for ASA_G
 //               then the ceil(N/n) global tokens in 128-row tiles.  Rows past N
@@ -9,7 +9,8 @@
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_j = Q K_j^T   (SS MMA, M=128 N=128) into TMEM S buffer j%2,
 //                 O_{j%2} += P_j V_j   (TS MMA: P read from TMEM, V from shared memory).
-//   warps 2..9  two softmax warpgroups.  Warpgroup w takes the tiles j = w, w+2, ...:
+//   warps 2, 3  idle (they complete warpgroup 0 for the register split)
+//   warps 4..11 two softmax warpgroups.  Warpgroup w takes the tiles j = w, w+2, ...:
 //               an independent online softmax (running max / sum in the log2 domain)
 //               with its own S buffer and its own O accumulator, so that one
 //               warpgroup's loads, reductions and stores overlap the other's exp2 work
@@ -32,7 +33,11 @@ namespace asa {
 
 namespace {
 
-constexpr int kFwdTcThreads = 320;  // producer, MMA, 2 softmax warpgroups
+constexpr int kFwdTcThreads = 384;  // warpgroup 0: producer, MMA; 1, 2: softmax streams
+// Register split (launch: 384 threads x 168 = 64,512 registers): warpgroup 0 gives
+// back to 72 per thread, the softmax warpgroups grow to 216.  128 x 72 + 256 x 216 =
+// 64,512; per sub-partition one warp of each warpgroup: 32 x (72 + 2 x 216) <= 16,384.
+constexpr uint32_t kRegsLow = 72, kRegsHigh = 216;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D, int NST>
@@ -62,6 +67,51 @@ __device__ __forceinline__ float exp2_fma(float x) {
   const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
                        9.999280572e-01f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
+
+// Blackwell paired fp32 arithmetic: two lanes of work per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_fma on a pair of lanes, the adds and the polynomial in paired arithmetic
+__device__ __forceinline__ void exp2_fma2(uint64_t x2, float& ea, float& eb) {
+  float xa, xb;
+  f2_unpack(x2, xa, xb);
+  xa = fmaxf(xa, -125.f);
+  xb = fmaxf(xb, -125.f);
+  const uint64_t x = f2_pack(xa, xb);
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t nmagic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t j = f2_add(x, magic);
+  const uint64_t n = f2_add(j, nmagic);
+  float na, nb;
+  f2_unpack(n, na, nb);
+  const uint64_t f = f2_add(x, f2_pack(-na, -nb));
+  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
+                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float pa, pb, ja, jb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(j, ja, jb);
+  ea = __int_as_float(__float_as_int(pa) + (__float_as_int(ja) << 23));
+  eb = __int_as_float(__float_as_int(pb) + (__float_as_int(jb) << 23));
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -158,6 +208,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   bool failed = false;
 
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producers
     // lane 0 streams Q and the K tiles, lane 1 the V tiles: a K stage is released as
@@ -204,15 +256,19 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idPV = tc::idesc_bf16(128, D, false, true);
+      // Descriptors are built once; an offset of `o` bytes into a tile adds o >> 4 to
+      // the start-address field (all tiles lie below 256 KB, so it never carries).
+      const uint64_t dQ = tc::sdesc_sw128(base + L::kQ, 16, 1024);
+      const uint64_t dK = tc::sdesc_sw128(base + L::kK, 16, 1024);
+      const uint64_t dV = tc::sdesc_sw128(base + L::kV, 16384, 1024);
       // S_j = Q K_j^T into S buffer j % 2
       auto issue_s = [&](int j) {
         const uint32_t dS = tmem + 128u * (j & 1);
-        const uint32_t kb = base + L::kK + (j % NST) * L::kTile;
+        const uint64_t kst = dK + (((j % NST) * L::kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-          tc::umma_ss(dS, tc::sdesc_sw128(base + L::kQ + off, 16, 1024),
-                      tc::sdesc_sw128(kb + off, 16, 1024), idS, ks > 0 ? 1u : 0u);
+          const uint32_t off = ((ks >> 2) * 16384u + (ks & 3) * 32u) >> 4;
+          tc::umma_ss(dS, dQ + off, kst + off, idS, ks > 0 ? 1u : 0u);
         }
       };
       bool ok = tc::mbar_wait(q_full(), 0, wait_limit);
@@ -238,10 +294,10 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         // O_b += P_j V_j; the first tile of a stream initialises its O
         const uint32_t tP = tmem + 128u * b;
         const uint32_t tO = tmem + 256u + 128u * b;
-        const uint32_t vb = base + L::kV + (j % NST) * L::kTile;
+        const uint64_t vst = dV + (((j % NST) * L::kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
-          tc::umma_ts(tO, tP + 8u * ks, tc::sdesc_sw128(vb + ks * 2048u, 16384, 1024), idPV,
+          tc::umma_ts(tO, tP + 8u * ks, vst + ((ks * 2048u) >> 4), idPV,
                       (j >= 2 || ks > 0) ? 1u : 0u);
         tc::umma_commit(v_empty(j % NST));
         tc::umma_commit(o_done(b));
@@ -259,11 +315,13 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         tc::mbar_wait(drain, 0, wait_limit);
       }
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     // ------------------------------------------------------------ softmax warpgroups
     // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
     // (wait results are AND-reduced over the warp).
-    const int w = (warp - 2) >> 2;  // stream: tiles w, w + 2, ...
+    const int w = (warp - 4) >> 2;  // stream: tiles w, w + 2, ...
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -312,24 +370,27 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       // P = exp2(s c2 + bias - m) packed to bf16 pairs (masked columns give exp2(-inf) = 0)
       const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
       uint32_t p[64];
-      float rs0 = 0.f, rs1 = 0.f;
+      const uint64_t c2x2 = f2_pack(c2, c2), offx2 = f2_pack(off, off);
+      uint64_t rs = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int k = 0; k < 64; ++k) {
-        const float xa = fmaf(__uint_as_float(s[2 * k]), c2, off);
-        const float xb = fmaf(__uint_as_float(s[2 * k + 1]), c2, off);
+        const uint64_t x2 =
+            f2_fma(f2_pack(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2x2, offx2);
         float a, bb;
         if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == 0) {
-          a = exp2_fma(xa);
-          bb = exp2_fma(xb);
+          exp2_fma2(x2, a, bb);
         } else {
+          float xa, xb;
+          f2_unpack(x2, xa, xb);
           a = fast_exp2(xa);
           bb = fast_exp2(xb);
         }
-        rs0 += a;
-        rs1 += bb;
+        rs = f2_add(rs, f2_pack(a, bb));
         p[k] = pack_bf16(a, bb);
       }
-      l = l * alpha + (rs0 + rs1);
+      float rsa, rsb;
+      f2_unpack(rs, rsa, rsb);
+      l = l * alpha + (rsa + rsb);
       if (it > 0) {
         // this stream's previous PV is done: O may be rescaled
         if (!wait_warp(o_done(w), (it - 1) & 1)) {
