@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "wan2.1-1.3b"
 METRIC = "ASA ms/call & effective TFLOP/s at 32760 tok, H=12, d=128, τ=0.95"
-KERNELS_PER_STEP = 8   # permute3, est_logits, est_pool, mask_rows, scan, fill, fwd, unpermute
+KERNELS_PER_STEP = 9   # permute3, est_logits, est_pool, mask_rows, scan, fill, lpt_order, fwd, unpermute
 
 
 def _peaks():
@@ -215,6 +215,7 @@ def main():
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     out = torch.empty_like(q)
     ws = asa.estimate_mask_workspace(B, H, N, dev)
+    fws = asa.fwd_workspace(B, H, N, d, 0, dev)
     mask = asa._alloc_mask(B, H, N, dev, transposed=False)
     stream = torch.cuda.current_stream()
 
@@ -229,7 +230,7 @@ def main():
         asa.asa_estimate_mask(qp, kp, wl.tau, transposed=False, workspace=ws, mask=mask)
         if marks is not None:
             marks[2].record(stream)
-        asa.asa_sparse_attn_fwd(qp, kp, vp, mask, out=op, lse=lse)
+        asa.asa_sparse_attn_fwd(qp, kp, vp, mask, workspace=fws, out=op, lse=lse)
         if marks is not None:
             marks[3].record(stream)
         asa.asa_unpermute(op, T, Hg, W, out=out)

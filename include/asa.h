@@ -158,7 +158,8 @@ int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d
  */
 int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n, void* stream);
 
-/* Workspace bytes of asa_sparse_attn_fwd (0 for standard ASA). */
+/* Workspace bytes of asa_sparse_attn_fwd: the launch order of the query blocks
+ * (longest kept list first), plus the global tokens for ASA_G. */
 size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window);
 
 /*

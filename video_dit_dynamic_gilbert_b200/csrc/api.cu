@@ -341,9 +341,14 @@ int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n,
 }
 
 size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window) {
-  if (global_window <= 0 || B < 1 || H < 1 || N < 1) return 0;
-  const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
-  return 2 * align256(static_cast<size_t>(B) * H * G * d * 2);
+  if (B < 1 || H < 1 || N < 1 || global_window < 0) return 0;
+  const size_t nb = (static_cast<size_t>(N) + ASA_BLOCK - 1) / ASA_BLOCK;
+  size_t bytes = align256(static_cast<size_t>(B) * H * nb * sizeof(int32_t));  // launch order
+  if (global_window > 0) {
+    const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    bytes += 2 * align256(static_cast<size_t>(B) * H * G * d * 2);
+  }
+  return bytes;
 }
 
 int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
@@ -365,9 +370,11 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const void* kg = nullptr;
   const void* vg = nullptr;
+  const size_t nb = (static_cast<size_t>(N) + ASA_BLOCK - 1) / ASA_BLOCK;
+  int32_t* order = static_cast<int32_t*>(workspace);
   if (global_window > 0) {
     const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
-    char* base = static_cast<char*>(workspace);
+    char* base = static_cast<char*>(workspace) + align256(static_cast<size_t>(B) * H * nb * sizeof(int32_t));
     void* kgw = base;
     void* vgw = base + align256(static_cast<size_t>(B) * H * G * d * 2);
     cudaError_t e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, num_sms_current(), s);
@@ -380,8 +387,8 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
   unsigned int* err_word = nullptr;
   cudaError_t e = device_error_word(&err_word);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
-  e = asa::launch_fwd_tc(qp, kp, vp, row_ptr, col_idx, kg, vg, B * H, N, d, global_window, o, lse,
-                         err_word, s);
+  e = asa::launch_fwd_tc(qp, kp, vp, row_ptr, col_idx, kg, vg, order, B * H, N, d, global_window, o,
+                         lse, err_word, s);
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
   return ASA_OK;
 }

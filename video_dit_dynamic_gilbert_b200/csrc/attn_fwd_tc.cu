@@ -152,16 +152,19 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
                   const __grid_constant__ CUtensorMap tmVg, const int32_t* __restrict__ row_ptr,
-                  const int32_t* __restrict__ col_idx, int N, int nb, int G, float gbias2,
-                  float c2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                  unsigned int* __restrict__ err_word, long long wait_limit) {
+                  const int32_t* __restrict__ col_idx, const int32_t* __restrict__ order, int N,
+                  int nb, int G, float gbias2, float c2, __nv_bfloat16* __restrict__ o,
+                  float* __restrict__ lse, unsigned int* __restrict__ err_word,
+                  long long wait_limit) {
   using L = FwdTcLayout<D, NST>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
 
-  const int I = blockIdx.x, bh = blockIdx.y;
+  // CTAs take query blocks in descending order of kept blocks (longest first)
+  const int rowid = order[blockIdx.x];
+  const int I = rowid % nb, bh = rowid / nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = I * kBlock;
   const int rbeg = row_ptr[bh * nb + I];
@@ -499,6 +502,49 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   }
 }
 
+// order[k] = the CSR row with the k-th largest number of kept blocks (counting sort
+// by count, one CTA).  Launching the longest query blocks first keeps the last wave
+// of the grid short.
+__global__ void __launch_bounds__(1024) lpt_order_kernel(const int32_t* __restrict__ row_ptr,
+                                                        int rows, int nb,
+                                                        int32_t* __restrict__ order) {
+  extern __shared__ int32_t start[];  // nb + 1 bins
+  __shared__ int32_t chunk_tot[1024];
+  const int tid = threadIdx.x;
+  for (int c = tid; c <= nb; c += blockDim.x) start[c] = 0;
+  __syncthreads();
+  for (int r = tid; r < rows; r += blockDim.x) atomicAdd(&start[row_ptr[r + 1] - row_ptr[r]], 1);
+  __syncthreads();
+  // exclusive scan over bins in descending count: bin c starts after all bins > c
+  const int nbins = nb + 1;
+  const int per = (nbins + blockDim.x - 1) / blockDim.x;
+  const int lo = tid * per, hi = min(nbins, lo + per);  // this thread's bins, reversed index
+  int32_t sum = 0;
+  for (int k = lo; k < hi; ++k) sum += start[nb - k];
+  chunk_tot[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int t = 0; t < static_cast<int>(blockDim.x); ++t) {
+      const int32_t v = chunk_tot[t];
+      chunk_tot[t] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  int32_t run = chunk_tot[tid];
+  for (int k = lo; k < hi; ++k) {
+    const int32_t v = start[nb - k];
+    start[nb - k] = run;
+    run += v;
+  }
+  __syncthreads();
+  for (int r = tid; r < rows; r += blockDim.x) {
+    const int c = row_ptr[r + 1] - row_ptr[r];
+    order[atomicAdd(&start[c], 1)] = r;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -528,7 +574,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
 
 template <int D, int NST>
 cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int32_t* col_idx,
-                      int BH, int N, int G, float gbias2, void* o, float* lse,
+                      int32_t* order, int BH, int N, int G, float gbias2, void* o, float* lse,
                       unsigned int* err_word, cudaStream_t stream) {
   using L = FwdTcLayout<D, NST>;
   const int nb = (N + kBlock - 1) / kBlock;
@@ -537,8 +583,12 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
-  fwd_tc_kernel<D, NST><<<dim3(nb, BH), kFwdTcThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, N, nb, G, gbias2, c2,
+  const int rows = nb * BH;
+  lpt_order_kernel<<<1, 1024, (nb + 1) * sizeof(int32_t), stream>>>(row_ptr, rows, nb, order);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  fwd_tc_kernel<D, NST><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, order, N, nb, G, gbias2, c2,
       static_cast<__nv_bfloat16*>(o), lse, err_word, limit);
   return cudaGetLastError();
 }
@@ -546,9 +596,9 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
 }  // namespace
 
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
-                          const int32_t* col_idx, const void* kg, const void* vg, int BH, int N,
-                          int d, int global_window, void* o, float* lse, unsigned int* err_word,
-                          cudaStream_t stream) {
+                          const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
+                          int BH, int N, int d, int global_window, void* o, float* lse,
+                          unsigned int* err_word, cudaStream_t stream) {
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
   const float gbias2 = global_window > 0 ? log2f(static_cast<float>(global_window)) : 0.f;
   CUtensorMap maps[5];
@@ -562,8 +612,9 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
     maps[3] = maps[1];
     maps[4] = maps[2];
   }
-  if (d == 128) return launch_tc<128, 3>(maps, row_ptr, col_idx, BH, N, G, gbias2, o, lse, err_word, stream);
-  return launch_tc<64, 6>(maps, row_ptr, col_idx, BH, N, G, gbias2, o, lse, err_word, stream);
+  if (d == 128)
+    return launch_tc<128, 3>(maps, row_ptr, col_idx, order, BH, N, G, gbias2, o, lse, err_word, stream);
+  return launch_tc<64, 6>(maps, row_ptr, col_idx, order, BH, N, G, gbias2, o, lse, err_word, stream);
 }
 
 }  // namespace asa

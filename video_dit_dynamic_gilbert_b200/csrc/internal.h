@@ -35,9 +35,9 @@ cudaError_t launch_fwd_mma(const void* qp, const void* kp, const void* vp, const
                            int d, int global_window, void* o, float* lse, cudaStream_t stream);
 
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
-                          const int32_t* col_idx, const void* kg, const void* vg, int BH, int N,
-                          int d, int global_window, void* o, float* lse, unsigned int* err_word,
-                          cudaStream_t stream);
+                          const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
+                          int BH, int N, int d, int global_window, void* o, float* lse,
+                          unsigned int* err_word, cudaStream_t stream);
 
 cudaError_t launch_bwd_mma(const void* qp, const void* kp, const void* vp, const void* o,
                            const void* dout, const float* lse, const int32_t* row_ptr,
