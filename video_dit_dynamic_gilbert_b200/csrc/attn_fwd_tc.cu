@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
 
-  // CTAs take query blocks in descending order of kept blocks (longest first)
+  // CTAs take the heads in order and, inside a head, the longest query blocks first
   const int rowid = order[blockIdx.x];
   const int I = rowid % nb, bh = rowid / nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -502,23 +502,25 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
   }
 }
 
-// order[k] = the CSR row with the k-th largest number of kept blocks (counting sort
-// by count, one CTA).  Launching the longest query blocks first keeps the last wave
-// of the grid short.
+// Launch order of the query blocks: heads in order (concurrent CTAs then share one
+// head's K and V in L2), and inside each head the query blocks with the most kept
+// blocks first, so that the grid ends on short CTAs.  One CTA per head: a counting
+// sort of its nb rows by kept-block count.
 __global__ void __launch_bounds__(1024) lpt_order_kernel(const int32_t* __restrict__ row_ptr,
-                                                        int rows, int nb,
-                                                        int32_t* __restrict__ order) {
+                                                        int nb, int32_t* __restrict__ order) {
   extern __shared__ int32_t start[];  // nb + 1 bins
   __shared__ int32_t chunk_tot[1024];
   const int tid = threadIdx.x;
+  const int r0 = blockIdx.x * nb;
   for (int c = tid; c <= nb; c += blockDim.x) start[c] = 0;
   __syncthreads();
-  for (int r = tid; r < rows; r += blockDim.x) atomicAdd(&start[row_ptr[r + 1] - row_ptr[r]], 1);
+  for (int r = tid; r < nb; r += blockDim.x)
+    atomicAdd(&start[row_ptr[r0 + r + 1] - row_ptr[r0 + r]], 1);
   __syncthreads();
   // exclusive scan over bins in descending count: bin c starts after all bins > c
   const int nbins = nb + 1;
   const int per = (nbins + blockDim.x - 1) / blockDim.x;
-  const int lo = tid * per, hi = min(nbins, lo + per);  // this thread's bins, reversed index
+  const int lo = min(nbins, tid * per), hi = min(nbins, lo + per);  // reversed bin index
   int32_t sum = 0;
   for (int k = lo; k < hi; ++k) sum += start[nb - k];
   chunk_tot[tid] = sum;
@@ -539,9 +541,9 @@ __global__ void __launch_bounds__(1024) lpt_order_kernel(const int32_t* __restri
     run += v;
   }
   __syncthreads();
-  for (int r = tid; r < rows; r += blockDim.x) {
-    const int c = row_ptr[r + 1] - row_ptr[r];
-    order[atomicAdd(&start[c], 1)] = r;
+  for (int r = tid; r < nb; r += blockDim.x) {
+    const int c = row_ptr[r0 + r + 1] - row_ptr[r0 + r];
+    order[r0 + atomicAdd(&start[c], 1)] = r0 + r;
   }
 }
 
@@ -584,7 +586,7 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   if (e != cudaSuccess) return e;
   const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
   const int rows = nb * BH;
-  lpt_order_kernel<<<1, 1024, (nb + 1) * sizeof(int32_t), stream>>>(row_ptr, rows, nb, order);
+  lpt_order_kernel<<<BH, 1024, (nb + 1) * sizeof(int32_t), stream>>>(row_ptr, nb, order);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   fwd_tc_kernel<D, NST><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
