@@ -42,6 +42,25 @@ def _peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def _fwd_traffic_bytes():
+    """dram read+write bytes per forward launch from the committed ncu summary, or None
+    when the kernel source has changed since that capture."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "fwd_tc_kernel_wan2.1-1.3b.md")
+    src = os.path.join(ROOT, "video_dit_dynamic_gilbert_b200", "csrc", "attn_fwd_tc.cu")
+    try:
+        txt = open(prof).read()
+        want = re.search(r"sha256 prefix\s+([0-9a-f]{16})", txt).group(1)
+        have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if want != have:
+            return None
+        mb = re.search(r"traffic per launch \(read \+ write\) \| ([0-9.]+) MB", txt).group(1)
+        return float(mb) * 1e6
+    except (OSError, AttributeError):
+        return None
+
+
 def _kept_tile_flops(row_ptr, col_idx, B, H, N, d):
     """4 d sum over kept (I, J) of L_I L_J, from the CSR the step produced."""
     nb = -(-N // 128)
@@ -288,7 +307,7 @@ def main():
         "effective_flops_per_call": flops,
         "roofline": {"kernel": "asa sparse attention forward", "bound": "tensor",
                      "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
-                     "frac": achieved / burst, "traffic": None,
+                     "frac": achieved / burst, "traffic": _fwd_traffic_bytes(),
                      "peak_kind": f"{peak_kind} bf16 burst",
                      "frac_of_sustained": achieved / sustained},
         "clocks": clk,
