@@ -131,8 +131,9 @@ int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* wor
  * as asa_estimate minus the workspace.
  *   - Scratch: one file-scope device array of ASA_NOALLOC_SCRATCH_BYTES, reserved on
  *     every device that loads the library and held until the process exits.  Shapes
- *     needing more (4 * B*H*16*nb*(nb+1) bytes) are rejected with ASA_ERR_WORKSPACE
- *     before anything is launched.
+ *     needing more (about 6.2 MB per head at N = 32,760 and d = 128, i.e. at most 5
+ *     heads per call at that shape) are rejected with ASA_ERR_WORKSPACE before
+ *     anything is launched.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
  *     capture.

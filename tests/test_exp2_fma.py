@@ -1,5 +1,5 @@
 """Error bound of the FMA-pipe exp2 used for a share of the softmax exponentials in
-the forward kernel (csrc/attn_fwd_tc.cu, exp2_fma): the float32 steps are emulated
+the tcgen05 kernels (csrc/softmax_math.cuh, exp2_fma): the float32 steps are emulated
 in NumPy and compared with exp2 in float64.  The bound (1e-4 relative) is well below
 the bf16 rounding (2^-8 relative step) that every P value gets right after."""
 import os
@@ -10,7 +10,7 @@ import sys
 import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-KERNEL = os.path.join(ROOT, "video_dit_dynamic_gilbert_b200", "csrc", "attn_fwd_tc.cu")
+KERNEL = os.path.join(ROOT, "video_dit_dynamic_gilbert_b200", "csrc", "softmax_math.cuh")
 GEN = os.path.join(ROOT, "video_dit_dynamic_gilbert_b200", "csrc", "gen_exp2_poly.py")
 
 

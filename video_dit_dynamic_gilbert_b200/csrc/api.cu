@@ -119,8 +119,7 @@ int check_ptr(const void* p, const char* name, bool need16 = true) {
   } while (0)
 
 struct MaskWs {
-  float* G;
-  float* lse2;
+  float* est;  // estimator scratch
   float* p_imp;
   uint8_t* bitmap;
   int32_t* counts;
@@ -136,7 +135,7 @@ MaskWs carve_mask_ws(void* base, int BH, int nb) {
     off += align256(n);
     return o;
   };
-  const size_t o_g = take(asa::est_scratch_floats(BH, nb) * sizeof(float));
+  const size_t o_g = take(asa::est_scratch_floats(BH, nb) * sizeof(float) + 256);
   const size_t o_p = take(static_cast<size_t>(BH) * nb * nb * sizeof(float));
   const size_t o_b = take(static_cast<size_t>(BH) * nb * nb);
   const size_t o_c = take(static_cast<size_t>(BH) * nb * sizeof(int32_t));
@@ -144,8 +143,7 @@ MaskWs carve_mask_ws(void* base, int BH, int nb) {
   w.bytes = off;
   if (base) {
     char* b = static_cast<char*>(base);
-    w.G = reinterpret_cast<float*>(b + o_g);
-    w.lse2 = w.G + static_cast<size_t>(BH) * nb * asa::kSamplesHost * nb;
+    w.est = reinterpret_cast<float*>(b + o_g);
     w.p_imp = reinterpret_cast<float*>(b + o_p);
     w.bitmap = reinterpret_cast<uint8_t*>(b + o_b);
     w.counts = reinterpret_cast<int32_t*>(b + o_c);
@@ -185,7 +183,7 @@ int record_error(int code, const char* fmt, ...) {
 }
 }  // namespace asa
 
-namespace {
+namespace asa {
 // Device address of g_device_error for the current device (kernels set bits in it
 // when a bounded wait expires).
 cudaError_t device_error_word(unsigned int** out) {
@@ -194,7 +192,8 @@ cudaError_t device_error_word(unsigned int** out) {
   *out = static_cast<unsigned int*>(p);
   return e;
 }
-}  // namespace
+}  // namespace asa
+using asa::device_error_word;
 
 extern "C" {
 
@@ -265,8 +264,11 @@ int asa_estimate(const void* qp, const void* kp, int B, int H, int N, int d, int
   const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
   MaskWs w = carve_mask_ws(workspace, B * H, nb);
   ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
-  cudaError_t e = asa::launch_estimate(qp, kp, B * H, N, d, w.G, w.lse2, p_imp, num_sms_current(),
-                                       static_cast<cudaStream_t>(stream));
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_estimate(qp, kp, B * H, N, d, w.est, p_imp, err_word, num_sms_current(),
+                           static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
   return ASA_OK;
 }
@@ -322,8 +324,11 @@ int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d
   const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
   MaskWs w = carve_mask_ws(workspace, B * H, nb);
   ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
-  cudaError_t e = asa::launch_estimate(qp, kp, B * H, N, d, w.G, w.lse2, w.p_imp, num_sms_current(),
-                                       static_cast<cudaStream_t>(stream));
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_estimate(qp, kp, B * H, N, d, w.est, w.p_imp, err_word, num_sms_current(),
+                           static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "estimate launch");
   return build_mask_impl(w.p_imp, B, H, N, tau, w, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t,
                          stream);

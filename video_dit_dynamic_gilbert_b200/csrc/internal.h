@@ -18,9 +18,15 @@ cudaError_t launch_permute(const void* const* src, void* const* dst, int ntensor
                            const int32_t* perm_dev, int B, int N, int H, int d, int num_sms,
                            cudaStream_t stream);
 
+// Estimator scratch (floats, 256-byte aligned base): G, lse2, per-chunk sums, Q_s, K_s.
 size_t est_scratch_floats(int BH, int nb);
-cudaError_t launch_estimate(const void* qp, const void* kp, int BH, int N, int d, float* G,
-                            float* lse2, float* p_imp, int num_sms, cudaStream_t stream);
+cudaError_t launch_estimate(const void* qp, const void* kp, int BH, int N, int d, float* scratch,
+                            float* p_imp, unsigned int* err_word, int num_sms,
+                            cudaStream_t stream);
+
+// Device address of the library's error word on the current device (bounded waits
+// that expire set bits in it: 1 = attention forward, 2 = estimator).
+cudaError_t device_error_word(unsigned int** out);
 
 cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uint8_t* bitmap,
                               int32_t* counts, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
