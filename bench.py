@@ -122,64 +122,99 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": n, "samples_under_load": len(sm)}
 
 
-def cpu_oracle_sample(wl, x, budget_s=15.0):
-    """Time the fp64 oracle on a bounded sample of the workload: estimate + mask of one
-    head, then the sparse forward of as many of its query blocks as fit the budget."""
+def oracle_setup(wl, x, h=0):
+    """The oracle's permuted Q, K, V of head h and its estimate + mask, with the time
+    the estimate + mask took."""
     import oracle
-    import threadpoolctl
     perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
-    h = 0
     t0 = time.perf_counter()
-    qp = oracle.permute(x["q"][:, :, h:h + 1].double().numpy(), perm)
-    kp = oracle.permute(x["k"][:, :, h:h + 1].double().numpy(), perm)
-    vp = oracle.permute(x["v"][:, :, h:h + 1].double().numpy(), perm)
+    qp, kp, vp = (oracle.permute(x[n][:, :, h:h + 1].double().numpy(), perm)
+                  for n in ("q", "k", "v"))
     pimp = oracle.estimate_pimp(qp, kp)
     mask = oracle.build_mask(pimp, wl.tau)
-    t_mask = time.perf_counter() - t0
+    return qp, kp, vp, mask, time.perf_counter() - t0
+
+
+def cpu_oracle_sample(wl, x, budget_s=15.0, setup=None, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload: estimate + mask of one
+    head (or the given `setup` of it), then the sparse forward of as many of its query
+    blocks as fit the budget.  The head's estimate + mask is charged in proportion to
+    the blocks sampled."""
+    import oracle
+    import threadpoolctl
+    qp, kp, vp, mask, t_mask = setup if setup is not None else oracle_setup(wl, x)
     nb = mask.shape[-1]
     flops, blocks, t_fwd = 0, 0, 0.0
     L = oracle.block_sizes(wl.N)
-    order = np.random.default_rng(0).permutation(nb)
+    order = np.random.default_rng(seed).permutation(nb)
     for I in order:
         t1 = time.perf_counter()
         oracle.asa_forward(qp, kp, vp, mask, q_index=np.arange(128 * I, 128 * I + L[I]))
         t_fwd += time.perf_counter() - t1
         flops += 4 * wl.d * L[I] * sum(L[J] for J in np.nonzero(mask[0, 0, I])[0])
         blocks += 1
-        if t_mask + t_fwd > budget_s:
+        if t_fwd + (t_mask if setup is None else 0.0) > budget_s:
             break
-    # the sample's per-head share of estimate+mask is charged in proportion
     t_total = t_fwd + t_mask * blocks / nb
     info = threadpoolctl.threadpool_info()
     cores = max([i.get("num_threads", 1) for i in info] or [1])
     return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds": t_total,
             "sample": (f"1 of {wl.H} heads: fp64 estimate+mask of the head ({t_mask:.1f} s, charged "
                        f"{blocks}/{nb} of it) + sparse forward of {blocks} of {nb} query blocks "
                        f"({t_fwd:.1f} s)")}
 
 
+def reference_step_budget(steps, warmup, total_s=150.0, cap_s=10.0):
+    """Seconds of oracle work per reference step, so that the whole run stays within a
+    few minutes whatever --steps and --warmup are."""
+    return max(0.2, min(cap_s, total_s / max(1, steps + warmup)))
+
+
 def run_reference(args, wl):
-    """The reference arm: the fp64 CPU oracle, timed as it stands, on a bounded sample."""
+    """The reference arm: the fp64 CPU oracle, timed as it stands, on a bounded sample
+    per step (rank 0 only; other ranks exit without work)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
-        return
+        return None
     from inputs import make_inputs
     x = make_inputs(wl)
+    setup = oracle_setup(wl, x)
+    budget = reference_step_budget(args.steps, args.warmup, cap_s=args.ref_budget)
     vals = []
     for step in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(wl, x, budget_s=args.ref_budget)
+        r = cpu_oracle_sample(wl, x, budget_s=budget, setup=setup, seed=step)
         if step >= args.warmup:
             vals.append(r)
     v = statistics.median(r["value"] for r in vals)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(r["seconds"] for r in vals),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(wl),
-        "cpu_baseline": {**vals[-1], "value": v},
+        "cpu_baseline": {**{k: vals[-1][k] for k in ("unit", "cores", "kind", "sample")},
+                         "value": v},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+    return line
+
+
+def rank_seed(wl, rank):
+    """Each rank runs its own independent seeded call (weak scaling)."""
+    return wl.seed + 1000 * rank
+
+
+def combine_over_ranks(dist, device, times, work):
+    """Max over ranks of each time in `times` and the sum over ranks of `work`: the
+    same two collectives on every rank, in the same order."""
+    import torch
+    t = torch.tensor([float(v) for v in times], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    dist.all_reduce(w)
+    return [float(v) for v in t.tolist()], float(w.item())
 
 
 def _config(wl):
@@ -225,7 +260,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    x = make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    x = make_inputs(wl.with_(seed=rank_seed(wl, rank)))
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
     B, N, H, d = q.shape
     T, Hg, W = wl.T, wl.Hg, wl.W
@@ -278,27 +313,15 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     elapsed_ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-        f = torch.tensor([float(flops)], device=dev, dtype=torch.float64)
-        dist.all_reduce(f)
-        total_flops = float(f.item())
-    else:
-        total_flops = float(flops)
-
-    ms_step = elapsed_ms / args.steps
     stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
     st_ms = stage.mean(axis=0)
     fwd_ms = float(st_ms[2])
-    value = total_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
 
     burst, sustained, hbm, peak_kind = _peaks()
     achieved = flops / (fwd_ms * 1e-3) / 1e12
     result = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "metric": METRIC, "value": None, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": _config(wl),
         "stages_ms": {"permute_qkv": float(st_ms[0]), "estimate_mask": float(st_ms[1]),
@@ -317,25 +340,32 @@ def main():
     # ---- end to end through the public call, host buffers in and out
     qh, kh, vh = (x[n].pin_memory() for n in ("q", "k", "v"))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    e_times = []
+    # device time on the launching stream, from the first H2D copy to the end of the D2H
+    e_ms = []
     for i in range(args.e2e_steps + 2):
+        e0, e1 = ev(), ev()
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
+        e0.record(stream)
         qd, kd, vd = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
         o_d, _, _ = asa.asa_attention(qd, kd, vd, T, Hg, W, wl.tau)
         oh.copy_(o_d, non_blocking=True)
+        e1.record(stream)
         torch.cuda.synchronize()
         if i >= 2:
-            e_times.append(time.perf_counter() - t0)
-    e_s = statistics.median(e_times)
+            e_ms.append(e0.elapsed_time(e1))
+    e_s = statistics.median(e_ms) * 1e-3
+
+    # whole job: max over ranks of each time, work summed over ranks
     if world > 1:
-        t = torch.tensor([e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_s = float(t.item())
+        (elapsed_ms, e_s), total_flops = combine_over_ranks(dist, dev, [elapsed_ms, e_s], flops)
+    else:
+        total_flops = float(flops)
+    result["ms_per_step"] = elapsed_ms / args.steps
+    result["value"] = total_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
     nbytes = q.numel() * q.element_size()
     result["e2e"] = {"value": total_flops / e_s / 1e12, "unit": "TFLOP/s",
                      "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
-                     "ms_per_call": e_s * 1e3}
+                     "ms_per_call": e_s * 1e3, "timing": "CUDA events on the stream"}
 
     if not args.no_extras:
         result["extras"] = extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream)

@@ -179,7 +179,11 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
                         int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
                         void* stream);
 
-/* Workspace bytes of asa_sparse_attn_bwd. */
+/*
+ * Workspace bytes of asa_sparse_attn_bwd (0 for invalid sizes): per-row lse*log2(e)
+ * and D (fp32, rows padded to whole blocks), fp16 copies of Q and K
+ * (2 * B*H*N*d * 2 bytes), and the launch orders of query and key blocks.
+ */
 size_t asa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
@@ -188,8 +192,11 @@ size_t asa_bwd_workspace_size(int B, int H, int N, int d);
  *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), dV = P^T dO, all over kept tiles only.
  * D equals rowsum(dO * O) in exact arithmetic; it is recomputed in fp32 from the kept
  * tiles because the bf16-rounded O would cost ~4e-3 relative L2 on dQ.  `o` is
- * validated but not read.  dS enters the dQ and dK products in fp16, so Q and K
- * magnitudes must stay below 65504.
+ * validated but not read.  dS enters the dQ and dK products in fp16 (so do Q and K,
+ * as fp16 copies in the workspace): Q and K magnitudes must stay at or below 65504;
+ * a larger value is reported by the next asa_check_device_status as
+ * ASA_ERR_INVALID_ARG (the gradients of that call are then meaningless).
+ * Deterministic: every output row is written by one CTA, without atomics.
  * qp, kp, vp, o, dout: device bf16 [B, H, N, d]; lse: device fp32 [B, H, N] from the
  * forward; row_ptr/col_idx and col_ptr_t/row_idx_t: both CSRs of asa_build_mask;
  * dq, dk, dv: device bf16 [B, H, N, d] (fully written; no accumulation into them).
@@ -204,7 +211,8 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of
  * the current device.  Returns ASA_OK, ASA_ERR_TIMEOUT if a kernel gave up a
- * bounded wait since the last check, or ASA_ERR_CUDA on a CUDA error.
+ * bounded wait since the last check, ASA_ERR_INVALID_ARG if a backward call met Q or
+ * K values beyond fp16 range, or ASA_ERR_CUDA on a CUDA error.
  */
 int asa_check_device_status(void* stream);
 

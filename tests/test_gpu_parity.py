@@ -160,6 +160,88 @@ def test_backward_with_oracle_mask(name):
     check_close(dq, rq, what="dQ")
     check_close(dk, rk, what="dK")
     check_close(dv, rv, what="dV")
+    asa.asa_check_device_status()
+
+
+def _backward_pair(name, mask, dout_scale=1.0):
+    """Library backward and oracle backward under a given mask [B, H, nb, nb]; dO is
+    multiplied by a power of two `dout_scale` (exact in bf16) on both sides."""
+    wl, x, perm, ref, pimp, _, marg, dev = setup_case(name)
+    dout = ref["dout"] * dout_scale
+    dq_d, dkv_d = oracle.asa_backward(ref["q"], ref["k"], ref["v"], dout, mask)
+    qp, kp, vp = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda() for k in ("q", "k", "v"))
+    dop = torch.from_numpy(dout).to(torch.bfloat16).cuda()
+    bm = upload_mask(mask, wl.N)
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
+    got = asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm)
+    asa.asa_check_device_status()
+    exp = [np.zeros(got[0].shape) for _ in range(3)]
+    for (bb, h, I), blk in dq_d.items():
+        exp[0][bb, h, 128 * I:128 * I + blk.shape[0]] = blk
+    for (bb, h, J), (gk, gv) in dkv_d.items():
+        exp[1][bb, h, 128 * J:128 * J + gk.shape[0]] = gk
+        exp[2][bb, h, 128 * J:128 * J + gv.shape[0]] = gv
+    return (qp, kp, vp, o, dop, lse, bm), got, exp
+
+
+@pytest.mark.parametrize("name", ["multi-tile", "d64-b2"])
+def test_backward_unkept_key_blocks(name):
+    """Rows keeping one block (their own) or two, and key blocks that no query block
+    keeps: those get dK = dV = 0 exactly.  Every query block keeps block 0, so its dV
+    sums thousands of dO rows; dO is scaled by 1/16 to keep the gradients O(1), where
+    the absolute bar is not swamped by the bf16 rounding of the output itself."""
+    wl = CASES[name]
+    nb = -(-wl.N // 128)
+    mask = np.zeros((wl.B, wl.H, nb, nb), dtype=bool)
+    for I in range(nb):
+        mask[:, :, I, I] = True
+    mask[:, :, :, 0] = True            # everyone keeps block 0
+    mask[:, :, 1, :] = False           # ... block 1 keeps only itself
+    mask[:, :, 1, 1] = True
+    mask[:, :, nb - 1, nb - 1] = False  # the last key block is kept by nobody
+    mask[:, :, nb - 1, 0] = True
+    args, got, exp = _backward_pair(name, mask, dout_scale=1.0 / 16)
+    for g, e, what in zip(got, exp, ("dQ", "dK", "dV")):
+        assert np.abs(e).max() < 2.0, (what, np.abs(e).max())
+        check_close(f64(g), e, what=what)
+    assert (f64(got[1])[:, :, 128 * (nb - 1):] == 0).all()
+    assert (f64(got[2])[:, :, 128 * (nb - 1):] == 0).all()
+
+
+@pytest.mark.parametrize("name", ["one-ragged-block", "d128-ragged"])
+def test_backward_dense_mask(name):
+    wl = CASES[name]
+    nb = -(-wl.N // 128)
+    mask = np.ones((wl.B, wl.H, nb, nb), dtype=bool)
+    _, got, exp = _backward_pair(name, mask)
+    for g, e, what in zip(got, exp, ("dQ", "dK", "dV")):
+        check_close(f64(g), e, what=what)
+
+
+def test_backward_deterministic():
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case("multi-tile")
+    args, got, _ = _backward_pair("multi-tile", mask)
+    again = asa.asa_sparse_attn_bwd(*args)
+    for a, b in zip(got, again):
+        assert torch.equal(a, b)
+
+
+def test_backward_reports_fp16_overflow():
+    """A Q value beyond fp16 range is reported by the next status check (the kernels
+    run to completion on the overflowed copy; nothing waits on it)."""
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case("tiny")
+    qp, kp, vp, dop = (torch.from_numpy(ref[k]).to(torch.bfloat16).cuda()
+                       for k in ("q", "k", "v", "dout"))
+    bm = upload_mask(mask, wl.N)
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
+    asa.asa_check_device_status()
+    qbad = qp.clone()
+    qbad[0, 0, 3, 5] = 70000.0
+    asa.asa_sparse_attn_bwd(qbad, kp, vp, o, dop, lse, bm)
+    with pytest.raises(asa.AsaError) as ei:
+        asa.asa_check_device_status()
+    assert ei.value.code == asa.ASA_ERR_INVALID_ARG
+    asa.asa_check_device_status()       # the word was cleared
 
 
 @pytest.mark.parametrize("name", ["tiny", "d64-b2", "multi-tile"])

@@ -399,9 +399,8 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
 }
 
 size_t asa_bwd_workspace_size(int B, int H, int N, int d) {
-  (void)d;
-  if (B < 1 || H < 1 || N < 1) return 0;
-  return 2 * align256(static_cast<size_t>(B) * H * N * sizeof(float));
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return asa::bwd_tc_workspace_bytes(B * H, N, d);
 }
 
 int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
@@ -422,12 +421,12 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
   ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
   const size_t need = asa_bwd_workspace_size(B, H, N, d);
   ASA_TRY(check_ws(workspace, ws_bytes, need));
-  float* Dvec = static_cast<float*>(workspace);
-  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         align256(static_cast<size_t>(B) * H * N * sizeof(float)));
-  cudaError_t e = asa::launch_bwd_mma(qp, kp, vp, o, dout, lse, row_ptr, col_idx, col_ptr_t,
-                                      row_idx_t, B * H, N, d, Dvec, lse2, dq, dk, dv,
-                                      num_sms_current(), static_cast<cudaStream_t>(stream));
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_bwd_tc(qp, kp, vp, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
+                         d, workspace, dq, dk, dv, err_word, num_sms_current(),
+                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return ASA_OK;
 }
@@ -441,6 +440,9 @@ int asa_check_device_status(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (word & 8u)
+      return fail(ASA_ERR_INVALID_ARG,
+                  "backward: a Q or K value is out of fp16 range (|x| > 65504) (word 0x%x)", word);
     return fail(ASA_ERR_TIMEOUT, "a device-side bounded wait expired (word 0x%x)", word);
   }
   return ASA_OK;

@@ -495,8 +495,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH][rows][D] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle, zero fill
-bool make_map(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
+// [BH][rows][D] 16-bit elements, boxes of 64 columns x 128 rows, 128-byte swizzle,
+// zero fill outside the tensor
+bool make_map_dtype(CUtensorMap* m, const void* ptr, int BH, int rows, int D,
+                    CUtensorMapDataType dtype) {
   auto enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
@@ -505,15 +507,29 @@ bool make_map(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
                            static_cast<cuuint64_t>(rows) * D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, dtype, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
+  return make_map_dtype(m, ptr, BH, rows, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 }  // namespace
 
 bool make_map_rows(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
   return make_map(m, ptr, BH, rows, D);
+}
+
+bool make_map_rows_f16(CUtensorMap* m, const void* ptr, int BH, int rows, int D) {
+  return make_map_dtype(m, ptr, BH, rows, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+}
+
+cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
+                             cudaStream_t stream) {
+  lpt_order_kernel<<<BH, 1024, (nb + 1) * sizeof(int32_t), stream>>>(ptr, nb, order);
+  return cudaGetLastError();
 }
 
 namespace {
@@ -530,8 +546,7 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   if (e != cudaSuccess) return e;
   const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
   const int rows = nb * BH;
-  lpt_order_kernel<<<BH, 1024, (nb + 1) * sizeof(int32_t), stream>>>(row_ptr, nb, order);
-  e = cudaGetLastError();
+  e = launch_lpt_order(row_ptr, BH, nb, order, stream);
   if (e != cudaSuccess) return e;
   fwd_tc_kernel<D, NST><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, order, N, nb, G, gbias2, c2,

@@ -45,6 +45,20 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
                           int BH, int N, int d, int global_window, void* o, float* lse,
                           unsigned int* err_word, cudaStream_t stream);
 
+// Launch order of the blocks of a CSR (ptr[BH * nb + 1], global offsets): heads in
+// order, inside each head the rows with the most entries first.
+cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
+                             cudaStream_t stream);
+
+// Backward workspace (bytes, 256-aligned pieces): lse2 and D [BH][nb*128] f32,
+// fp16 copies of Q and K [BH][N][d], launch orders of query and key blocks [BH*nb].
+size_t bwd_tc_workspace_bytes(int BH, int N, int d);
+cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const void* dout,
+                          const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
+                          const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
+                          int d, void* workspace, void* dq, void* dk, void* dv,
+                          unsigned int* err_word, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_bwd_mma(const void* qp, const void* kp, const void* vp, const void* o,
                            const void* dout, const float* lse, const int32_t* row_ptr,
                            const int32_t* col_idx, const int32_t* col_ptr_t,
