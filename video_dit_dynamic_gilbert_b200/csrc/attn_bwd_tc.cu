@@ -12,7 +12,7 @@
 // the blocks with the most partners first):
 //   bwd_prep        fp16 copies of Q and K, lse2 (rows past N: +inf, so P = 0 there),
 //                   D cleared.  fp16 holds every bf16 value of magnitude in
-//                   [2^-17, 65504] exactly; a value that overflows sets bit 8 of the
+//                   [2^-17, 65504] exactly; a value that overflows ORs 8 into the
 //                   device error word.
 //   bwd_row<D pass> per query block I, walking its CSR row: S and dP into TMEM,
 //                   D_I = rowsum(P o dP) exactly in fp32.  (D from the bf16-rounded O
@@ -46,7 +46,7 @@
 // have read yet; the MMA reading them takes K-steps 0-3 from [0,32) and 4-7 from
 // [64,96) of the buffer.  A buffer is rewritten by the next MMA only after the MMA that
 // reads the packed operand, in issue order.  Every wait is bounded: on expiry the
-// kernel sets bit 4 of the device error word, drains its copies and MMAs, frees TMEM
+// kernel ORs 4 into the device error word, drains its copies and MMAs, frees TMEM
 // and returns.
 #include <cudaTypedefs.h>
 

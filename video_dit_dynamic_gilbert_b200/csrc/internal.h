@@ -36,10 +36,6 @@ cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uin
 cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, int n, int num_sms,
                                cudaStream_t stream);
 
-cudaError_t launch_fwd_mma(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
-                           const int32_t* col_idx, const void* kg, const void* vg, int BH, int N,
-                           int d, int global_window, void* o, float* lse, cudaStream_t stream);
-
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
                           const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
                           int BH, int N, int d, int global_window, void* o, float* lse,
@@ -58,12 +54,5 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, void* workspace, void* dq, void* dk, void* dv,
                           unsigned int* err_word, int num_sms, cudaStream_t stream);
-
-cudaError_t launch_bwd_mma(const void* qp, const void* kp, const void* vp, const void* o,
-                           const void* dout, const float* lse, const int32_t* row_ptr,
-                           const int32_t* col_idx, const int32_t* col_ptr_t,
-                           const int32_t* row_idx_t, int BH, int N, int d, float* Dvec,
-                           float* lse2, void* dq, void* dk, void* dv, int num_sms,
-                           cudaStream_t stream);
 
 }  // namespace asa
