@@ -223,6 +223,202 @@ def _config(wl):
             "l2": "inputs larger than L2: raster Q, K, V are 3 x 100.6 MB",
             "parallelism": "one independent call per GPU (weak)"}
 
+# ----------------------------------------------------------------------- measurement report
+
+def _near_threshold_rows(p_imp, tau, eps=1e-4, gap=1e-6):
+    """Mask rows whose cut is within `eps` of tau (or whose last kept and first dropped
+    shares differ by less than `gap`): the rows where fp32 and fp64 may cut differently."""
+    p = np.asarray(p_imp, dtype=np.float64).reshape(-1, p_imp.shape[-1])
+    r = -np.sort(-(p / p.sum(axis=1, keepdims=True)), axis=1)
+    cum = np.cumsum(r, axis=1)
+    c = np.minimum(np.argmax(cum >= tau, axis=1), r.shape[1] - 1)
+    rows = np.arange(len(c))
+    near = np.abs(cum[rows, c] - tau) < eps
+    near |= (c > 0) & (np.abs(cum[rows, np.maximum(c - 1, 0)] - tau) < eps)
+    nxt = np.minimum(c + 1, r.shape[1] - 1)
+    near |= (c + 1 < r.shape[1]) & (np.abs(r[rows, c] - r[rows, nxt]) < gap)
+    return int(near.sum()), int(len(c))
+
+
+class _Timer:
+    """Per-call CUDA-event times on one stream: median and min over `reps` calls after
+    `warm` untimed ones; `flush` (an L2-sized write) runs before each call, outside its
+    events."""
+
+    def __init__(self, torch, stream, flush_bytes=256 << 20):
+        self.torch, self.stream = torch, stream
+        self.buf = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+
+    def flush(self):
+        self.buf.fill_(1)
+
+    def __call__(self, fn, reps=20, warm=5, flush=False):
+        torch = self.torch
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            if flush:
+                self.flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return {"median_ms": float(statistics.median(ts)), "min_ms": float(min(ts))}
+
+
+def _report_config(asa, torch, wl, timer, dev, peaks):
+    """Every stage of one workload, timed separately (SURVEY-style split)."""
+    from inputs import make_inputs
+    x = make_inputs(wl, with_dout=wl.backward)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    B, N, H, d = q.shape
+    T, Hg, W = wl.T, wl.Hg, wl.W
+    nb = -(-N // 128)
+    qp, kp, vp = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    asa.asa_gilbert_permute3(q, k, v, T, Hg, W, outs=(qp, kp, vp))
+    ws = asa.estimate_mask_workspace(B, H, N, dev)
+    p_imp = torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
+    mask = asa._alloc_mask(B, H, N, dev, transposed=wl.backward)
+    gw = wl.global_window
+    fws = asa.fwd_workspace(B, H, N, d, gw, dev)
+    op = torch.empty_like(qp)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    tensor_bytes = q.numel() * q.element_size()
+    burst, sustained, hbm, kind = peaks
+    r = {"workload": wl.name, "B": B, "H": H, "N": N, "d": d, "tau": wl.tau, "global_window": gw}
+
+    def hbm_stage(name, fn, nbytes):
+        for fl in (True, False):
+            t = timer(fn, flush=fl)
+            t["GB_s"] = nbytes / (t["median_ms"] * 1e-3) / 1e9
+            t["frac_of_measured_hbm"] = t["GB_s"] / hbm
+            r[name + ("_l2_flushed" if fl else "_l2_warm")] = t
+
+    hbm_stage("permute_qkv", lambda: asa.asa_gilbert_permute3(q, k, v, T, Hg, W, outs=(qp, kp, vp)),
+              3 * 2 * tensor_bytes)
+    r["estimate"] = timer(lambda: asa.asa_estimate(qp, kp, workspace=ws, out=p_imp))
+    r["mask"] = timer(lambda: asa.asa_build_mask(p_imp, N, wl.tau, transposed=wl.backward,
+                                                 workspace=ws, mask=mask))
+    r["estimate_mask"] = timer(lambda: asa.asa_estimate_mask(qp, kp, wl.tau, transposed=wl.backward,
+                                                             workspace=ws, mask=mask))
+    torch.cuda.synchronize()
+    Ls = np.array([min(128, N - 128 * i) for i in range(nb)])
+    M = int(np.minimum(16, Ls).sum())
+    est_flops = 2 * M * M * d * B * H
+    r["estimate"]["TFLOP_s"] = est_flops / (r["estimate"]["median_ms"] * 1e-3) / 1e12
+    r["estimate"]["exp_count"] = M * M * B * H
+    near, rows = _near_threshold_rows(p_imp.cpu().numpy(), wl.tau)
+    r["near_threshold_rows"] = {"count": near, "of": rows}
+    flops, nnz, tiles = _kept_tile_flops(mask.row_ptr.cpu().numpy(), mask.col_idx.cpu().numpy(),
+                                         B, H, N, d)
+    r["kept_tiles"], r["tiles"], r["kept_fraction"] = nnz, tiles, nnz / tiles
+    if gw > 0:
+        G = -(-N // gw)
+        kg = torch.empty((B, H, G, d), dtype=torch.bfloat16, device=dev)
+        hbm_stage("pool_K", lambda: asa.asa_global_pool(kp, gw, out=kg),
+                  tensor_bytes + B * H * G * d * 2)
+        flops += 4 * d * N * G * B * H
+    r["effective_flops"] = flops
+    r["attn_fwd"] = timer(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=gw,
+                                                          workspace=fws, out=op, lse=lse))
+    t = r["attn_fwd"]["median_ms"] * 1e-3
+    r["attn_fwd"].update({"TFLOP_s": flops / t / 1e12, "frac_of_burst": flops / t / 1e12 / burst,
+                          "frac_of_sustained": flops / t / 1e12 / sustained,
+                          "frac_of_datasheet_2250": flops / t / 1e12 / 2250.0})
+    hbm_stage("unpermute_o", lambda: asa.asa_unpermute(op, T, Hg, W, out=out), 2 * tensor_bytes)
+    em = r["estimate_mask"]["median_ms"]
+    r["estimate_mask_share"] = em / (em + r["attn_fwd"]["median_ms"])
+    if wl.backward:
+        do = x["dout"].to(dev)
+        dop = asa.asa_gilbert_permute(do, T, Hg, W)
+        bws = asa.bwd_workspace(B, H, N, d, dev)
+        grads = tuple(torch.empty_like(qp) for _ in range(3))
+        r["attn_bwd"] = timer(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, mask,
+                                                              workspace=bws, outs=grads),
+                              reps=8, warm=3)
+        tb = r["attn_bwd"]["median_ms"] * 1e-3
+        r["attn_bwd"]["effective_TFLOP_s"] = 2.5 * flops / tb / 1e12
+        r["attn_bwd"]["executed_TFLOP_s"] = 4.5 * flops / tb / 1e12
+    asa.asa_check_device_status()
+    return r, (qp, kp, vp)
+
+
+def _dense(asa, torch, timer, qp, kp, vp, peaks):
+    """Dense attention on the same inputs: our kernel with every tile kept, and torch SDPA."""
+    B, H, N, d = qp.shape
+    nb = -(-N // 128)
+    dense_flops = 4 * d * N * N * B * H
+    full = asa.asa_build_mask(torch.ones((B, H, nb, nb), dtype=torch.float32, device=qp.device),
+                              N, 1.0, transposed=False)
+    ours = timer(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, full), reps=10, warm=3)
+    sdpa = timer(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp),
+                 reps=10, warm=3)
+    burst = peaks[0]
+    for t in (ours, sdpa):
+        t["TFLOP_s"] = dense_flops / (t["median_ms"] * 1e-3) / 1e12
+        t["frac_of_burst"] = t["TFLOP_s"] / burst
+    return {"ours_tau1": ours, "torch_sdpa": sdpa, "dense_flops": dense_flops}
+
+
+def run_report(path):
+    """Every measurement of the scope table, one JSON file: per-stage times of each
+    workload (median and min of 20 CUDA-event-timed calls after 5 warm-up calls; the
+    copy kernels with and without an L2 flush), dense comparisons, the tau sweep on the
+    CogVideoX-5B shape and the backward on the Wan-14B shape."""
+    import torch
+    from inputs import WORKLOADS, make_inputs
+    from video_dit_dynamic_gilbert_b200 import asa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    timer = _Timer(torch, stream)
+    peaks = _peaks()
+    rep = {"peaks": {"bf16_burst_tflops": peaks[0], "bf16_sustained_tflops": peaks[1],
+                     "hbm_gbs": peaks[2], "kind": peaks[3]},
+           "device": torch.cuda.get_device_name(dev), "configs": {}, "dense": {}, "tau_sweep": []}
+    clocks = ClockSampler(0)
+    for name in ("tiny", "wan2.1-1.3b", "cogvideox-5b", "wan2.1-1.3b-asag", "wan-14b-720p"):
+        wl = WORKLOADS[name]
+        r, (qp, kp, vp) = _report_config(asa, torch, wl, timer, dev, peaks)
+        rep["configs"][name] = r
+        if name in ("wan2.1-1.3b", "cogvideox-5b"):
+            rep["dense"][name] = _dense(asa, torch, timer, qp, kp, vp, peaks)
+        if name == "cogvideox-5b":
+            B, H, N, d = qp.shape
+            ws = asa.estimate_mask_workspace(B, H, N, dev)
+            for tau in (0.80, 0.90, 0.95, 0.99):
+                m = asa.asa_estimate_mask(qp, kp, tau, transposed=False, workspace=ws)
+                em = timer(lambda: asa.asa_estimate_mask(qp, kp, tau, transposed=False,
+                                                         workspace=ws, mask=m))
+                fw = timer(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, m))
+                flops, nnz, tiles = _kept_tile_flops(m.row_ptr.cpu().numpy(),
+                                                     m.col_idx.cpu().numpy(), B, H, N, d)
+                rep["tau_sweep"].append({
+                    "workload": name, "tau": tau, "kept_fraction": nnz / tiles,
+                    "estimate_mask": em, "attn_fwd": fw,
+                    "TFLOP_s": flops / (fw["median_ms"] * 1e-3) / 1e12,
+                    "estimate_mask_share": em["median_ms"] / (em["median_ms"] + fw["median_ms"])})
+        del qp, kp, vp
+        torch.cuda.empty_cache()
+    rep["clocks"] = clocks.stop()
+    with open(path, "w") as f:
+        json.dump(rep, f, indent=1)
+    for name, r in rep["configs"].items():
+        line = (f"{name:18s} fwd {r['attn_fwd']['median_ms']:.3f} ms "
+                f"{r['attn_fwd']['TFLOP_s']:.0f} TF/s ({r['attn_fwd']['frac_of_burst']:.3f} burst) "
+                f"est+mask {r['estimate_mask']['median_ms']:.3f} ms "
+                f"({100 * r['estimate_mask_share']:.1f}%) kept {r['kept_fraction']:.3f} "
+                f"perm {r['permute_qkv_l2_flushed']['GB_s']:.0f} GB/s")
+        if "attn_bwd" in r:
+            line += (f" bwd {r['attn_bwd']['median_ms']:.2f} ms "
+                     f"{r['attn_bwd']['effective_TFLOP_s']:.0f} TF/s eff")
+        print(line)
+    return rep
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -235,11 +431,16 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=10.0)
+    ap.add_argument("--report", metavar="PATH", default=None,
+                    help="run the full measurement set on one GPU, write it to PATH as JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from inputs import WORKLOADS, make_inputs
     wl = WORKLOADS[args.workload]
+    if args.report:
+        run_report(args.report)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
         return
