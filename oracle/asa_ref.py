@@ -8,7 +8,8 @@ Video Generation" (arXiv 2508.10774), section "Adaptive Block-Sparse Attention":
   * "Step 2.2: Computation", variant 1 (standard ASA) and variant 2 (ASA_G, global
     tokens with the fixed additive ln(n) mask)      -> asa_forward
   * the mask also restricts attention "during both training and inference" (end
-    of Step 2.1)                                    -> asa_backward (fixed mask)
+    of Step 2.1)                                    -> asa_backward (fixed mask; ASA
+    and ASA_G)
   * "Implementation details": b = 128, k = 16.
 
 Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
@@ -26,7 +27,10 @@ Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
     [n g, min(n g + n, N)), rounded to bf16 (the kernels store bf16 operands);
     every query sees every global token with logit q.kg / sqrt(d) + ln(n), also
     for the ragged last window;
-  * LSE is the natural-log log-sum-exp of the logits a query row attends to.
+  * LSE is the natural-log log-sum-exp of the logits a query row attends to;
+  * in the ASA_G backward the gradient of a global token reaches the rows of its
+    window through the mean (divided by the window's row count); its bf16 rounding
+    passes gradients unchanged.
 """
 from __future__ import annotations
 
@@ -258,19 +262,25 @@ def asa_forward(qp, kp, vp, mask, b: int = 128, global_window: int = 0,
 
 
 def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
-                 q_blocks=None, kv_blocks=None):
-    """Gradients of standard ASA under a fixed mask (the mask is not differentiated).
+                 q_blocks=None, kv_blocks=None, global_window: int = 0):
+    """Gradients of ASA under a fixed mask (the mask is not differentiated).
 
-    For each query block I with kept keys K_I, V_I:
-        P = softmax(Q_I K_I^T / sqrt(d)),  dV_I += P^T dO_I,  dP = dO_I V_I^T,
-        dS = P * (dP - rowsum(P * dP)),    dQ_I = dS K_I / sqrt(d),
-        dK_I += dS^T Q_I / sqrt(d).
+    For each query block I with kept keys K_I, V_I (and, for ASA_G, the global tokens
+    Kg, Vg of global_tokens() with the fixed + ln(n) on their logits):
+        P = softmax(logits),  dP = dO_I [V_I; Vg]^T,  dS = P * (dP - rowsum(P * dP)),
+        dQ_I = dS [K_I; Kg] / sqrt(d),
+        dK_J += dS_J^T Q_I / sqrt(d),  dV_J += P_J^T dO_I   (kept fine blocks J),
+        dKg += dS_g^T Q_I / sqrt(d),   dVg += P_g^T dO_I    (global tokens).
+    A global token is the mean of the n permuted rows of its window, so its gradient
+    reaches each of those rows divided by the window's row count (the bf16 rounding of
+    the pooled token passes gradients through unchanged).
     Returns dicts {(b, h, I): dQ block} and {(b, h, J): (dK block, dV block)} for
     the requested heads / blocks (all by default).
     """
     B, H, N, d = qp.shape
     nb = -(-N // b)
     scale = 1.0 / math.sqrt(d)
+    n = global_window
     heads = [(bb, h) for bb in range(B) for h in range(H)] if heads is None else list(heads)
     dq_out, dkv_out = {}, {}
     for (bb, h) in heads:
@@ -278,9 +288,14 @@ def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
         want_kv = set(range(nb)) if kv_blocks is None else set(kv_blocks)
         dK = {J: np.zeros((min(b, N - b * J), d)) for J in want_kv}
         dV = {J: np.zeros((min(b, N - b * J), d)) for J in want_kv}
+        if n > 0:
+            Kg = global_tokens(kp[bb, h], n)
+            Vg = global_tokens(vp[bb, h], n)
+            dKg = np.zeros_like(Kg)
+            dVg = np.zeros_like(Vg)
         for I in range(nb):
             kept = np.nonzero(mask[bb, h, I])[0]
-            if I not in want_q and not (set(kept.tolist()) & want_kv):
+            if n == 0 and I not in want_q and not (set(kept.tolist()) & want_kv):
                 continue
             rows = np.arange(b * I, min(b * I + b, N))
             idx = _kept_positions(mask[bb, h, I], N, b)
@@ -289,6 +304,11 @@ def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
             V = np.asarray(vp[bb, h, idx], dtype=np.float64)
             dO = np.asarray(dout[bb, h, rows], dtype=np.float64)
             S = (Q @ K.T) * scale
+            nf = len(idx)
+            if n > 0:
+                S = np.concatenate([S, (Q @ Kg.T) * scale + math.log(n)], axis=1)
+                K = np.concatenate([K, Kg], axis=0)
+                V = np.concatenate([V, Vg], axis=0)
             E = np.exp(S - S.max(axis=1, keepdims=True))
             P = E / E.sum(axis=1, keepdims=True)
             dP = dO @ V.T
@@ -302,6 +322,16 @@ def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
                     dK[J] += (dS[:, off:off + LJ].T @ Q) * scale
                     dV[J] += P[:, off:off + LJ].T @ dO
                 off += LJ
+            if n > 0:
+                dKg += (dS[:, nf:].T @ Q) * scale
+                dVg += P[:, nf:].T @ dO
+        if n > 0:
+            # MeanPool_n: row i of window g receives the window's gradient / its count
+            cnt = np.array([min(n, N - n * g) for g in range(len(Kg))], dtype=np.float64)
+            for J in want_kv:
+                r = np.arange(b * J, min(b * J + b, N))
+                dK[J] += dKg[r // n] / cnt[r // n, None]
+                dV[J] += dVg[r // n] / cnt[r // n, None]
         for J in want_kv:
             dkv_out[(bb, h, J)] = (dK[J], dV[J])
     return dq_out, dkv_out

@@ -118,10 +118,10 @@ def test_asa_g_window_one_doubles_kept_keys():
     np.testing.assert_allclose(O, ref.numpy(), rtol=1e-10, atol=1e-12)
 
 
-def _full_grads(q, k, v, dout, mask, b):
+def _full_grads(q, k, v, dout, mask, b, n=0):
     B, H, N, d = q.shape
     nb = mask.shape[2]
-    dq_d, dkv_d = oracle.asa_backward(q, k, v, dout, mask, b=b)
+    dq_d, dkv_d = oracle.asa_backward(q, k, v, dout, mask, b=b, global_window=n)
     dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
     for (bb, h, I), blk in dq_d.items():
         dq[bb, h, b * I:b * I + blk.shape[0]] = blk
@@ -174,6 +174,57 @@ def test_backward_finite_differences():
             num = (loss(args_p["q"], args_p["k"], args_p["v"])
                    - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
             assert abs(num - grad[0, 0, i, c]) < 1e-6 * max(1.0, abs(num)), (name, i, c)
+
+
+@pytest.mark.parametrize("N,n", [(300, 64), (256, 16), (200, 1)])
+def test_asa_g_backward_equals_autograd(N, n):
+    """ASA_G backward against torch autograd through SDPA over the augmented keys: the
+    global tokens are avg_pool1d windows of K and V (ragged last window over its own
+    count), rounded to bf16 by a straight-through step (value rounded, gradient
+    passed), with the fixed + ln(n) on their logits."""
+    B, H, d, b = 1, 2, 16, 128
+    q, k, v = (oracle.round_to_bf16(a) for a in _rand(B, H, N, d, 40 + N + n))
+    dout = np.random.default_rng(n).standard_normal(q.shape)
+    nb = -(-N // b)
+    g = np.random.default_rng(N)
+    mask = g.random((B, H, nb, nb)) < 0.5
+    mask[..., np.arange(nb), np.arange(nb)] = True
+    dq, dk, dv = _full_grads(q, k, v, dout, mask, b, n=n)
+
+    tq, tk, tv = (torch.from_numpy(a).requires_grad_(True) for a in (q, k, v))
+
+    def pool(x):
+        t = x.reshape(B * H, N, d).transpose(1, 2)
+        p = F.avg_pool1d(t, kernel_size=n, stride=n, ceil_mode=True)
+        p = p.transpose(1, 2).reshape(B, H, -1, d)
+        return p + (p.float().bfloat16().double() - p).detach()
+
+    Kg, Vg = pool(tk), pool(tv)
+    G = Kg.shape[2]
+    fine = torch.where(torch.from_numpy(_token_mask(mask, N, b)), 0.0, -math.inf).double()
+    bias = torch.cat([fine, torch.full((B, H, N, G), math.log(n), dtype=torch.float64)], dim=3)
+    O = F.scaled_dot_product_attention(tq, torch.cat([tk, Kg], dim=2), torch.cat([tv, Vg], dim=2),
+                                       attn_mask=bias)
+    O.backward(torch.from_numpy(dout))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_asa_g_backward_block_selection_matches_full():
+    B, H, N, d, b, n = 1, 1, 300, 8, 128, 64
+    q, k, v = (oracle.round_to_bf16(a) for a in _rand(B, H, N, d, 93))
+    dout = np.random.default_rng(4).standard_normal(q.shape)
+    mask = np.array([[[[1, 0, 0], [0, 1, 0], [1, 0, 1]]]], dtype=bool)
+    full_q, full_kv = oracle.asa_backward(q, k, v, dout, mask, b=b, global_window=n)
+    part_q, part_kv = oracle.asa_backward(q, k, v, dout, mask, b=b, heads=[(0, 0)],
+                                          q_blocks=[1], kv_blocks=[1], global_window=n)
+    np.testing.assert_allclose(part_q[(0, 0, 1)], full_q[(0, 0, 1)], rtol=1e-13)
+    # key block 1 is kept only by query block 1, but every query reaches it through
+    # the global tokens
+    np.testing.assert_allclose(part_kv[(0, 0, 1)][0], full_kv[(0, 0, 1)][0], rtol=1e-13)
+    np.testing.assert_allclose(part_kv[(0, 0, 1)][1], full_kv[(0, 0, 1)][1], rtol=1e-13)
+    assert np.abs(full_kv[(0, 0, 1)][1]).max() > 0
 
 
 def test_backward_block_selection_matches_full():
