@@ -126,10 +126,6 @@ struct Bars {
 };
 static_assert(10 + 2 * kNA + 2 * kNB == BwdLayout<128>::kNumBars, "barrier count");
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // the warp's tcgen05 loads/stores are complete: one arrive per warp
 __device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
   tc::fence_before();
@@ -141,10 +137,6 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
 // apart, the 16-element steps inside a half 32 bytes apart (descriptor units: >> 4)
 __device__ __forceinline__ uint32_t kmajor_step(int ks) {
   return ((ks >> 2) * 16384u + (ks & 3) * 32u) >> 4;
-}
-// K-step ks of a packed 128-wide TMEM operand written by the two warpgroups
-__device__ __forceinline__ uint32_t packed_step(int ks) {
-  return ks < 4 ? 8u * ks : 64u + 8u * (ks - 4);
 }
 
 // TMA side, warp 0: lane 0 the stationary tiles and ring A, lane 1 ring B.  Ring tile t
@@ -302,7 +294,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t kst = dKm + (((t % kNA) * L::kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
-          tc::umma_ts(tmem + 384u, tmem + 128u * (t & 1) + packed_step(ks),
+          tc::umma_ts(tmem + 384u, tmem + 128u * (t & 1) + tc::packed_half_step(ks),
                       kst + ((ks * 2048u) >> 4), idQ, (t > 0 || ks > 0) ? 1u : 0u);
       };
       bool ok = tc::mbar_wait(br.stat_full(), 0, wait_limit);
@@ -428,9 +420,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       f2_unpack(dsum2, da, db);
       const float part = da + db;
       float* red = reinterpret_cast<float*>(sbase + L::kStat0);
-      named_bar_sync(1, 256);
+      tc::named_bar_sync(1, 256);
       if (w == 1) red[row] = part;
-      named_bar_sync(1, 256);
+      tc::named_bar_sync(1, 256);
       if (w == 0 && q < N) Dvec[vrow] = part + red[row];
     } else {
       bool have = n > 0 && !failed;
@@ -543,14 +535,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t ost = dOm + (((t % kNB) * L::kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
-          tc::umma_ts(tmem + 256u, tmem + packed_step(ks), ost + ((ks * 2048u) >> 4), idV,
+          tc::umma_ts(tmem + 256u, tmem + tc::packed_half_step(ks), ost + ((ks * 2048u) >> 4), idV,
                       (t > 0 || ks > 0) ? 1u : 0u);
       };
       auto issue_dK = [&](int t) {  // dK += dS^T_t Q_t (the 1/sqrt(d) comes in the epilogue)
         const uint64_t qst = dQm + (((t % kNA) * L::kTile) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kBlock / 16; ++ks)
-          tc::umma_ts(tmem + 384u, tmem + 128u + packed_step(ks), qst + ((ks * 2048u) >> 4), idK,
+          tc::umma_ts(tmem + 384u, tmem + 128u + tc::packed_half_step(ks), qst + ((ks * 2048u) >> 4), idK,
                       (t > 0 || ks > 0) ? 1u : 0u);
       };
       bool ok = tc::mbar_wait(br.stat_full(), 0, wait_limit);

@@ -38,7 +38,12 @@ constexpr int kFwdTcThreads = 384;  // warpgroup 0: producer, MMA; 1, 2: softmax
 // Register split (launch: 384 threads x 168 = 64,512 registers): warpgroup 0 gives
 // back to 72 per thread, the softmax warpgroups grow to 216.  128 x 72 + 256 x 216 =
 // 64,512; per sub-partition one warp of each warpgroup: 32 x (72 + 2 x 216) <= 16,384.
+// The launcher checks the compiled count: a split above the launch allocation would
+// wait forever.
+constexpr int kLaunchRegs = 168;
 constexpr uint32_t kRegsLow = 72, kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh == kFwdTcThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 
 template <int D, int NST>
@@ -56,13 +61,11 @@ struct FwdTcLayout {
   static constexpr uint32_t kSmem = kBytes + 1024;  // + alignment slack
 };
 
-// One in kPolyEvery P pairs takes exp2_fma (0: all on MUFU).  A single softmax warp
-// reaches only ~2.8 of MUFU's 4 exp2/clk per sub-partition; the FMA pipe has room.
-constexpr int kPolyEvery = 4;
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
+// One in kPolyEvery(D) P pairs takes exp2_fma (0: all on MUFU).  A single softmax warp
+// reaches only part of MUFU's 4 exp2/clk per sub-partition; measured best: one pair in
+// 4 at d=64 (the tile is exponential-bound), one in 8 at d=128.
+template <int D>
+constexpr int poly_every() { return D == 128 ? 8 : 4; }
 
 struct TileSrc {
   int row0, nvalid;
@@ -316,6 +319,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         const uint64_t x2 =
             f2_fma(f2_pack(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2x2, offx2);
         float a, bb;
+        constexpr int kPolyEvery = poly_every<D>();
         if (kPolyEvery > 0 && (k % (kPolyEvery > 0 ? kPolyEvery : 1)) == 0) {
           exp2_fma2(x2, a, bb);
         } else {
@@ -370,11 +374,11 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     // merge the two streams: (m, l) through shared memory, over Q's bytes (every MMA
     // that reads Q is complete once both warpgroups hold their last PV)
     float* red = reinterpret_cast<float*>(sbase + L::kQ);  // [2][2][128]: m, l per stream
-    named_bar_sync(1, 256);
+    tc::named_bar_sync(1, 256);
     red[(2 * w) * 128 + row] = have_o ? m_ref : -INFINITY;
     red[(2 * w + 1) * 128 + row] = have_o ? l : 0.f;
     red[(4 + w) * 128 + row] = have_o ? 1.f : 0.f;
-    named_bar_sync(1, 256);
+    tc::named_bar_sync(1, 256);
     const float m_0 = red[0 * 128 + row], l_0 = red[1 * 128 + row];
     const float m_1 = red[2 * 128 + row], l_1 = red[3 * 128 + row];
     const bool has_0 = red[4 * 128 + row] != 0.f, has_1 = red[5 * 128 + row] != 0.f;
@@ -544,6 +548,15 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
+  // the register split inside the kernel assumes exactly kLaunchRegs per thread at launch
+  static int regs_checked = 0;
+  if (regs_checked == 0) {
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<D, NST>);
+    if (e != cudaSuccess) return e;
+    regs_checked = fa.numRegs == kLaunchRegs ? 1 : -1;
+  }
+  if (regs_checked < 0) return cudaErrorInvalidConfiguration;
   const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
   const int rows = nb * BH;
   e = launch_lpt_order(row_ptr, BH, nb, order, stream);
