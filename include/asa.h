@@ -182,14 +182,22 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
 /*
  * Workspace bytes of asa_sparse_attn_bwd (0 for invalid sizes): per-row lse*log2(e)
  * and D (fp32, rows padded to whole blocks), fp16 copies of Q and K
- * (2 * B*H*N*d * 2 bytes), and the launch orders of query and key blocks.
+ * (2 * B*H*N*d * 2 bytes), and the launch orders of query and key blocks; with
+ * global_window = n > 0 also the G = ceil(N/n) global tokens (bf16 K, V and fp16 K,
+ * B*H*G*d each) and their fp32 gradients (2 * B*H*G*d * 4 bytes).
  */
-size_t asa_bwd_workspace_size(int B, int H, int N, int d);
+size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window);
 
 /*
- * Backward of standard ASA under the fixed mask (the mask is not differentiated):
+ * Backward of ASA under the fixed mask (Video-BLADE, "Step 2.1": the mask restricts
+ * attention "during both training and inference"; it is not differentiated):
  *   P = exp(S - LSE), dP = dO V^T, D = rowsum(P * dP), dS = P * (dP - D),
  *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), dV = P^T dO, all over kept tiles only.
+ * global_window = n > 0: the backward of ASA_G ("Step 2.2", variant 2, the forward
+ * with the same n): the softmax also spans the G = ceil(N/n) global tokens (mean of
+ * K and V over each window of n permuted rows, logits + ln(n)); dQ gains their term,
+ * and the gradient of each global token reaches the rows of its window divided by
+ * the window's row count (its bf16 rounding passes gradients unchanged).
  * D equals rowsum(dO * O) in exact arithmetic; it is recomputed in fp32 from the kept
  * tiles because the bf16-rounded O would cost ~4e-3 relative L2 on dQ.  `o` is
  * validated but not read.  dS enters the dQ and dK products in fp16 (so do Q and K,
@@ -205,8 +213,8 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
                         const void* dout, const float* lse, const int32_t* row_ptr,
                         const int32_t* col_idx, const int32_t* col_ptr_t,
                         const int32_t* row_idx_t, int B, int H, int N, int d, int block,
-                        void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
-                        void* stream);
+                        int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
+                        void* dv, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of

@@ -295,7 +295,9 @@ def asa_backward(qp, kp, vp, dout, mask, b: int = 128, heads=None,
             dVg = np.zeros_like(Vg)
         for I in range(nb):
             kept = np.nonzero(mask[bb, h, I])[0]
-            if n == 0 and I not in want_q and not (set(kept.tolist()) & want_kv):
+            # every query block reaches every requested key block through the global
+            # tokens; without globals only through its kept blocks
+            if I not in want_q and not (want_kv if n > 0 else set(kept.tolist()) & want_kv):
                 continue
             rows = np.arange(b * I, min(b * I + b, N))
             idx = _kept_positions(mask[bb, h, I], N, b)

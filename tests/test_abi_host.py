@@ -118,8 +118,13 @@ def test_attention_rejects(L):
                                  FAKE, FAKE, None) == asa.ASA_ERR_WORKSPACE
     assert L.asa_sparse_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 64, 128, -1, None, 0,
                                  FAKE, FAKE, None) == asa.ASA_ERR_INVALID_ARG
-    args = [FAKE] * 10 + [1, 2, 1024, 64, 128, None, 0] + [FAKE] * 3 + [None]
+    args = [FAKE] * 10 + [1, 2, 1024, 64, 128, 0, None, 0] + [FAKE] * 3 + [None]
     assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_WORKSPACE
+    args[15] = -1    # global_window
+    assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_INVALID_ARG
+    args[15] = 64
+    assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_WORKSPACE
+    args[15] = 0
     args[9] = None   # row_idx_t
     assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_INVALID_ARG
 
@@ -130,5 +135,10 @@ def test_workspace_sizes(L):
     assert est >= 12 * nb * nb * (16 * 4 + 4 + 1)
     assert L.asa_fwd_workspace_size(1, 12, 32760, 128, 0) >= 12 * 256 * 4      # launch order
     assert L.asa_fwd_workspace_size(1, 12, 32760, 128, 64) >= 2 * 12 * 512 * 128 * 2
-    assert L.asa_bwd_workspace_size(1, 12, 32760, 128) >= 2 * 12 * 32760 * 4
+    assert L.asa_bwd_workspace_size(1, 12, 32760, 128, 0) >= 2 * 12 * 32760 * 4
+    # ASA_G adds the global tokens (bf16 K, V, fp16 K) and their fp32 gradients
+    G = -(-32760 // 64)
+    extra = L.asa_bwd_workspace_size(1, 12, 32760, 128, 64) - L.asa_bwd_workspace_size(1, 12, 32760, 128, 0)
+    assert extra >= 12 * G * 128 * (3 * 2 + 2 * 4)
+    assert L.asa_bwd_workspace_size(1, 12, 32760, 128, -1) == 0
     assert L.asa_estimate_mask_workspace_size(0, 12, 32760) == 0

@@ -127,3 +127,42 @@ def test_full_size_backward_wan14b():
     rows = slice(128 * J, min(128 * J + 128, wl.N))
     check_close(f64(dk[0, h, rows]), dkv_ref[(0, 0, J)][0], what=f"dK block {J}")
     check_close(f64(dv[0, h, rows]), dkv_ref[(0, 0, J)][1], what=f"dV block {J}")
+
+
+def test_full_size_backward_asa_g_wan():
+    """ASA_G backward at the Wan2.1-1.3B shape (n = 64), the bench's launch: the
+    invariants sum_j dV_j = sum_i dO_i and sum_j dK_j = 0 per head (rows of P over fine
+    and global keys sum to one and a window's rows share its token's gradient equally;
+    rows of dS sum to zero), and dQ of sampled query blocks of one head against the
+    oracle (a query block's dQ needs only its own row of the mask)."""
+    wl = WORKLOADS["wan2.1-1.3b-asag"]
+    n = wl.global_window
+    x = make_inputs(wl, with_dout=True)
+    perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
+    q, k, v, do = (x[name].cuda() for name in ("q", "k", "v", "dout"))
+    qp, kp, vp, dop = (asa.asa_gilbert_permute(t, wl.T, wl.Hg, wl.W) for t in (q, k, v, do))
+    h = 3
+    qh, kh, vh, doh = (_head(x, name, perm, h) for name in ("q", "k", "v", "dout"))
+    mask_h = oracle.build_mask(oracle.estimate_pimp(qh, kh), wl.tau)
+    full = mask_from_csr(asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True))
+    full[:, h] = mask_h[:, 0]
+    bm = upload_mask(full, wl.N)
+    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm, global_window=n)
+    dq, dk, dv = asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm, global_window=n)
+    torch.cuda.synchronize()
+    asa.asa_check_device_status()
+    sum_dv = dv.double().sum(dim=2)
+    sum_do = dop.double().sum(dim=2)
+    scale = dop.double().abs().sum(dim=2).clamp_min(1.0)
+    assert float(((sum_dv - sum_do).abs() / scale).max()) < 2e-2
+    kscale = dk.double().abs().sum(dim=2).clamp_min(1.0)
+    assert float((dk.double().sum(dim=2).abs() / kscale).max()) < 2e-2
+    g = np.random.default_rng(13)
+    nb = mask_h.shape[-1]
+    q_blocks = sorted(set(g.choice(nb - 1, 3, replace=False).tolist() + [nb - 1]))
+    dq_ref, _ = oracle.asa_backward(qh, kh, vh, doh, mask_h, heads=[(0, 0)], q_blocks=q_blocks,
+                                    kv_blocks=[], global_window=n)
+    for I in q_blocks:
+        rows = slice(128 * I, min(128 * I + 128, wl.N))
+        check_close(f64(dq[0, h, rows]), dq_ref[(0, 0, I)], what=f"ASA_G dQ block {I}")
+

@@ -41,8 +41,8 @@ _SIGNATURES = {
     "asa_global_pool": ([_vp, _vp] + [_c_int] * 5 + [_vp], _c_int),
     "asa_fwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
-    "asa_bwd_workspace_size": ([_c_int] * 4, _c_size),
-    "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 5 + [_vp, _c_size] + [_vp] * 4, _c_int),
+    "asa_bwd_workspace_size": ([_c_int] * 5, _c_size),
+    "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_shutdown": ([], None),
 }
@@ -270,25 +270,27 @@ def asa_sparse_attn_fwd(qp, kp, vp, mask: BlockMask, global_window: int = 0, wor
     return out, lse
 
 
-def bwd_workspace(B, H, N, d, device):
-    return _workspace(lib().asa_bwd_workspace_size(B, H, N, d), device)
+def bwd_workspace(B, H, N, d, device, global_window: int = 0):
+    return _workspace(lib().asa_bwd_workspace_size(B, H, N, d, global_window), device)
 
 
-def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, workspace=None, outs=None,
-                        stream=None):
-    """dQ, dK, dV [B, H, N, d] bf16 under the fixed mask (standard ASA)."""
+def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, global_window: int = 0,
+                        workspace=None, outs=None, stream=None):
+    """dQ, dK, dV [B, H, N, d] bf16 under the fixed mask (ASA; ASA_G with the forward's
+    global_window)."""
     for n_, t in (("qp", qp), ("kp", kp), ("vp", vp), ("o", o), ("dout", dout)):
         _bf16_cuda(n_, t)
     if mask.col_ptr_t is None:
         raise ValueError("the backward needs the transposed CSR (transposed=True)")
     B, H, N, d = qp.shape
     if workspace is None:
-        workspace = bwd_workspace(B, H, N, d, qp.device)
+        workspace = bwd_workspace(B, H, N, d, qp.device, global_window)
     if outs is None:
         outs = tuple(torch.empty_like(qp) for _ in range(3))
     _check(lib().asa_sparse_attn_bwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(o), _ptr(dout), _ptr(lse),
                                      _ptr(mask.row_ptr), _ptr(mask.col_idx), _ptr(mask.col_ptr_t),
-                                     _ptr(mask.row_idx_t), B, H, N, d, BLOCK, _ptr(workspace),
+                                     _ptr(mask.row_idx_t), B, H, N, d, BLOCK, global_window,
+                                     _ptr(workspace),
                                      workspace.numel(), *(_ptr(t) for t in outs), _stream(stream)))
     return outs
 

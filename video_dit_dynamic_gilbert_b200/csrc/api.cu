@@ -398,17 +398,17 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
   return ASA_OK;
 }
 
-size_t asa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  return asa::bwd_tc_workspace_bytes(B * H, N, d);
+size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128) || global_window < 0) return 0;
+  return asa::bwd_tc_workspace_bytes(B * H, N, d, global_window);
 }
 
 int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
                         const void* dout, const float* lse, const int32_t* row_ptr,
                         const int32_t* col_idx, const int32_t* col_ptr_t,
                         const int32_t* row_idx_t, int B, int H, int N, int d, int block,
-                        void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
-                        void* stream) {
+                        int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
+                        void* dv, void* stream) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_block(block, ASA_SAMPLES));
   const void* bf[] = {qp, kp, vp, o, dout, dq, dk, dv};
@@ -419,13 +419,14 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
   ASA_TRY(check_ptr(col_idx, "col_idx", false));
   ASA_TRY(check_ptr(col_ptr_t, "col_ptr_t", false));
   ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
-  const size_t need = asa_bwd_workspace_size(B, H, N, d);
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  const size_t need = asa_bwd_workspace_size(B, H, N, d, global_window);
   ASA_TRY(check_ws(workspace, ws_bytes, need));
   unsigned int* err_word = nullptr;
   cudaError_t e = device_error_word(&err_word);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
   e = asa::launch_bwd_tc(qp, kp, vp, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
-                         d, workspace, dq, dk, dv, err_word, num_sms_current(),
+                         d, global_window, workspace, dq, dk, dv, err_word, num_sms_current(),
                          static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return ASA_OK;

@@ -63,8 +63,13 @@ bool make_map_rows_f16(CUtensorMap* m, const void* ptr, int BH, int rows, int D)
 namespace {
 
 constexpr int kBwdThreads = 384;
-// 384 threads x 168 registers at launch; 128 x 72 + 256 x 216 = 64,512 (the forward's split)
+// 384 threads x 168 registers at launch; 128 x 72 + 256 x 216 = 64,512 (the forward's
+// split).  The launcher checks the compiled count: a split above the launch allocation
+// would wait forever.
+constexpr int kLaunchRegs = 168;
 constexpr uint32_t kRegsLow = 72, kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh == kBwdThreads * kLaunchRegs,
+              "register split must equal the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kNA = 3, kNB = 2;  // ring stages
 constexpr int kElemWarps = 8;
@@ -139,13 +144,16 @@ __device__ __forceinline__ uint32_t kmajor_step(int ks) {
   return ((ks >> 2) * 16384u + (ks & 3) * 32u) >> 4;
 }
 
-// TMA side, warp 0: lane 0 the stationary tiles and ring A, lane 1 ring B.  Ring tile t
-// is the 128-row block idx[t] of mA / mB.  Stage s of ring A is refilled after the
-// a_empty(s) commit of its previous tile, likewise for B.
+// TMA side, warp 0: lane 0 the stationary tiles and ring A, lane 1 ring B.  Ring tile
+// t < nfirst is the 128-row block idx[t] (t itself when idx is null) of mA / mB; tile
+// t >= nfirst is the 128-row tile t - nfirst of mA2 / mB2 (the ASA_G global tokens).
+// Stage s of ring A is refilled after the a_empty(s) commit of its previous tile,
+// likewise for B.
 template <int D>
 __device__ bool produce(const Bars& br, uint32_t base, int lane, const CUtensorMap* m0,
                         const CUtensorMap* m1, int row_stat, const CUtensorMap* mA,
-                        const CUtensorMap* mB, const int32_t* idx, int n, int bh,
+                        const CUtensorMap* mB, const int32_t* idx, int nfirst,
+                        const CUtensorMap* mA2, const CUtensorMap* mB2, int n, int bh,
                         long long limit) {
   using L = BwdLayout<D>;
   const bool isA = lane == 0;
@@ -172,12 +180,14 @@ __device__ bool produce(const Bars& br, uint32_t base, int lane, const CUtensorM
       ok = false;
       break;
     }
+    const bool second = t >= nfirst;
+    const int row = second ? (t - nfirst) * kBlock : (idx != nullptr ? idx[t] : t) * kBlock;
+    const CUtensorMap* m = isA ? (second ? mA2 : mA) : (second ? mB2 : mB);
     const uint32_t full = isA ? br.a_full(st) : br.b_full(st);
     tc::mbar_expect_tx(full, L::kTile);
 #pragma unroll
     for (int h = 0; h < D / 64; ++h)
-      tc::tma_load_3d(ring + st * L::kTile + h * 16384u, isA ? mA : mB, 64 * h, idx[t] * kBlock,
-                      bh, full);
+      tc::tma_load_3d(ring + st * L::kTile + h * 16384u, m, 64 * h, row, bh, full);
     issued = t + 1;
   }
   // every issued copy has landed and its stage has been released before the CTA exits
@@ -228,10 +238,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_row_kernel(const __grid_constant__ CUtensorMap tmQ16,
                    const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ CUtensorMap tmK16,
-                   const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ row_ptr,
+                   const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmKg16,
+                   const __grid_constant__ CUtensorMap tmVg, const int32_t* __restrict__ row_ptr,
                    const int32_t* __restrict__ col_idx, const int32_t* __restrict__ order, int N,
-                   int nb, int Np, float c2, float scale, const float* __restrict__ lse2,
-                   float* __restrict__ Dvec, __nv_bfloat16* __restrict__ dq,
+                   int nb, int Np, int G, float gbias2, float c2, float scale,
+                   const float* __restrict__ lse2, float* __restrict__ Dvec,
+                   __nv_bfloat16* __restrict__ dq,
                    unsigned int* __restrict__ err_word, long long wait_limit) {
   using L = BwdLayout<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -244,7 +257,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = I * kBlock;
   const int rbeg = row_ptr[bh * nb + I];
-  const int n = row_ptr[bh * nb + I + 1] - rbeg;
+  const int nfine = row_ptr[bh * nb + I + 1] - rbeg;
+  const int n = nfine + (G > 0 ? (G + kBlock - 1) / kBlock : 0);  // + ASA_G global tiles
   const int32_t* cols = col_idx + rbeg;
 
   const Bars br{base + L::kBars};
@@ -264,7 +278,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
       if (lane < 2)
-        failed = !produce<D>(br, base, lane, &tmQ16, &tmdO, q0, &tmK16, &tmV, cols, n, bh,
+        failed = !produce<D>(br, base, lane, &tmQ16, &tmdO, q0, &tmK16, &tmV, cols, nfine, &tmKg16,
+                             &tmVg, n, bh,
                              wait_limit);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
@@ -377,9 +392,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::tmem_wait_ld_dep32(s + 32);
       if (kDPass) warp_arrive(br.ds_full(t & 1), lane);
       float p[64];
-      exp2_64(s, c2, [&](int) { return nl2; }, p);
-      // key columns past N (the ragged last block) get no weight
-      const int nvalid = min(kBlock, N - cols[t] * kBlock) - 64 * w;
+      // global tokens carry + ln(n) (log2(n) in these units)
+      const bool glob = t >= nfine;
+      const float off = nl2 + (glob ? gbias2 : 0.f);
+      exp2_64(s, c2, [&](int) { return off; }, p);
+      // key columns past N (the ragged last block) or past G get no weight
+      const int nvalid = (glob ? min(kBlock, G - (t - nfine) * kBlock)
+                               : min(kBlock, N - cols[t] * kBlock)) - 64 * w;
       if (nvalid < 64) {
 #pragma unroll
         for (int k = 0; k < 64; ++k)
@@ -462,30 +481,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ------------------------------------------------------------------ key-block kernel
 
-template <int D>
+// kGlobal = false: one CTA per fine key block J, walking the query blocks that keep J
+// (transposed CSR); with ASA_G (gw > 0) the epilogue adds each row's share of its
+// window's global-token gradient, dKg[g] / count_g and dVg[g] / count_g, before the
+// single bf16 rounding.
+// kGlobal = true (ASA_G): one CTA per 128 global tokens, walking every query block
+// (every query attends to every global token, logits + ln(n)); writes dKg (with the
+// 1/sqrt(d)) and dVg in fp32.
+template <int D, bool kGlobal>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_col_kernel(const __grid_constant__ CUtensorMap tmK16,
                    const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ16,
                    const __grid_constant__ CUtensorMap tmdO, const int32_t* __restrict__ col_ptr_t,
                    const int32_t* __restrict__ row_idx_t, const int32_t* __restrict__ order,
-                   int N, int nb, int Np, float c2, float scale, const float* __restrict__ lse2,
-                   const float* __restrict__ Dvec, __nv_bfloat16* __restrict__ dk,
-                   __nv_bfloat16* __restrict__ dv, unsigned int* __restrict__ err_word,
-                   long long wait_limit) {
+                   int N, int nb, int Np, int G, int gw, float gbias2, float c2, float scale,
+                   const float* __restrict__ lse2, const float* __restrict__ Dvec,
+                   __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                   float* __restrict__ dKg32, float* __restrict__ dVg32,
+                   unsigned int* __restrict__ err_word, long long wait_limit) {
   using L = BwdLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
 
-  const int colid = order[blockIdx.x];
-  const int J = colid % nb, bh = colid / nb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k0 = J * kBlock;
-  const int cbeg = col_ptr_t[bh * nb + J];
-  const int n = col_ptr_t[bh * nb + J + 1] - cbeg;
-  const int32_t* rows = row_idx_t + cbeg;
+  int bh, k0, n;
+  const int32_t* rows;
+  if constexpr (kGlobal) {
+    const int ng = (G + kBlock - 1) / kBlock;
+    bh = blockIdx.x / ng;
+    k0 = (blockIdx.x % ng) * kBlock;  // first global token of the tile
+    n = nb;
+    rows = nullptr;                   // query block t at step t
+  } else {
+    const int colid = order[blockIdx.x];
+    const int J = colid % nb;
+    bh = colid / nb;
+    k0 = J * kBlock;
+    const int cbeg = col_ptr_t[bh * nb + J];
+    n = col_ptr_t[bh * nb + J + 1] - cbeg;
+    rows = row_idx_t + cbeg;
+  }
 
   const Bars br{base + L::kBars};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kTmemSlot);
@@ -504,7 +542,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
       if (lane < 2)
-        failed = !produce<D>(br, base, lane, &tmK16, &tmV, k0, &tmQ16, &tmdO, rows, n, bh,
+        failed = !produce<D>(br, base, lane, &tmK16, &tmV, k0, &tmQ16, &tmdO, rows, n, &tmQ16,
+                             &tmdO, n, bh,
                              wait_limit);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
@@ -605,18 +644,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool ok = tc::mbar_wait(bar, parity, wait_limit);
       return __all_sync(0xffffffffu, ok) != 0;
     };
+    const float bias = kGlobal ? gbias2 : 0.f;  // global tokens: + ln(n) in log2 units
     for (int t = 0; t < n; ++t) {
       // the query tile's lse2 and D (same addresses across the warp: broadcast loads)
-      const float4* lv = reinterpret_cast<const float4*>(l2h + rows[t] * kBlock);
-      const float4* dvv = reinterpret_cast<const float4*>(ddh + rows[t] * kBlock);
+      const int qb = kGlobal ? t : rows[t];
+      const float4* lv = reinterpret_cast<const float4*>(l2h + qb * kBlock);
+      const float4* dvv = reinterpret_cast<const float4*>(ddh + qb * kBlock);
       float off[64];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const float4 v = __ldg(lv + c);
-        off[4 * c] = -v.x;
-        off[4 * c + 1] = -v.y;
-        off[4 * c + 2] = -v.z;
-        off[4 * c + 3] = -v.w;
+        off[4 * c] = bias - v.x;
+        off[4 * c + 1] = bias - v.y;
+        off[4 * c + 2] = bias - v.z;
+        off[4 * c + 3] = bias - v.w;
       }
       if (!wait_warp(br.s_full(0), t & 1)) {
         failed = true;
@@ -671,19 +712,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     // warpgroup 0 writes dV, warpgroup 1 dK (scaled by 1/sqrt(d)); a key block that no
-    // query block keeps gets zeros
-    __nv_bfloat16* drow = (w == 0 ? dv : dk) + (static_cast<int64_t>(bh) * N + (kr < N ? kr : 0)) * D;
+    // query block keeps gets zeros (plus, with ASA_G, its global share)
     const float f = w == 0 ? 1.f : scale;
+    if constexpr (kGlobal) {
+      float* grow = (w == 0 ? dVg32 : dKg32) + (static_cast<int64_t>(bh) * G + (kr < G ? kr : 0)) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t a[32];
-      if (have) {
-        tc::tmem_ld32_sync(trow + 256u + 128u * w + 32u * c, a);
-      } else {
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        if (have) {
+          tc::tmem_ld32_sync(trow + 256u + 128u * w + 32u * c, a);
+        } else {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) a[k] = 0u;
+          for (int k = 0; k < 32; ++k) a[k] = 0u;
+        }
+        if (kr < G) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<float4*>(grow + 32 * c + 4 * v) =
+                make_float4(__uint_as_float(a[4 * v]) * f, __uint_as_float(a[4 * v + 1]) * f,
+                            __uint_as_float(a[4 * v + 2]) * f, __uint_as_float(a[4 * v + 3]) * f);
+        }
       }
-      if (kr < N) store_row_bf16(drow + 32 * c, a, f);
+    } else {
+      __nv_bfloat16* drow =
+          (w == 0 ? dv : dk) + (static_cast<int64_t>(bh) * N + (kr < N ? kr : 0)) * D;
+      // the row's window in the global tokens (ASA_G): its gradient / the window's rows
+      const float* gsrc = nullptr;
+      float ginv = 0.f;
+      if (gw > 0 && kr < N) {
+        const int g = kr / gw;
+        gsrc = (w == 0 ? dVg32 : dKg32) + (static_cast<int64_t>(bh) * G + g) * D;
+        ginv = 1.f / static_cast<float>(min(gw, N - g * gw));
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        if (have) {
+          tc::tmem_ld32_sync(trow + 256u + 128u * w + 32u * c, a);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] = 0u;
+        }
+        if (kr < N) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] = __float_as_uint(__uint_as_float(a[k]) * f);
+          if (gsrc != nullptr) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 gv = *reinterpret_cast<const float4*>(gsrc + 32 * c + 4 * v);
+              a[4 * v] = __float_as_uint(fmaf(gv.x, ginv, __uint_as_float(a[4 * v])));
+              a[4 * v + 1] = __float_as_uint(fmaf(gv.y, ginv, __uint_as_float(a[4 * v + 1])));
+              a[4 * v + 2] = __float_as_uint(fmaf(gv.z, ginv, __uint_as_float(a[4 * v + 2])));
+              a[4 * v + 3] = __float_as_uint(fmaf(gv.w, ginv, __uint_as_float(a[4 * v + 3])));
+            }
+          }
+          store_row_bf16(drow + 32 * c, a, 1.f);
+        }
+      }
     }
   }
 
@@ -729,92 +814,186 @@ __global__ void __launch_bounds__(256)
   if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0) atomicOr(err_word, kErrRange);
 }
 
+// fp16 copy of a bf16 tensor (8 elements per step; overflow ORs kErrRange)
+__global__ void __launch_bounds__(256)
+    f16_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n8,
+                    unsigned int* __restrict__ err_word) {
+  uint32_t bad = 0;
+  auto cvt = [&](uint32_t v) {
+    const uint32_t h = bf16x2_to_f16x2(v);
+    bad |= ((h & 0x7c00u) == 0x7c00u) | ((h & 0x7c000000u) == 0x7c000000u);
+    return h;
+  };
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n8;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 a = src[j];
+    dst[j] = make_uint4(cvt(a.x), cvt(a.y), cvt(a.z), cvt(a.w));
+  }
+  if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0) atomicOr(err_word, kErrRange);
+}
+
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace pieces (256-byte aligned, in this order): lse2, D [BH][nb*128] f32; Q16,
+// K16 [BH][N][d] f16; launch orders of query and key blocks [BH*nb] i32; with ASA_G
+// (G global tokens): Kg, Vg [BH][G][d] bf16, Kg16 [BH][G][d] f16, dKg, dVg [BH][G][d] f32.
+struct BwdWs {
+  float *lse2, *Dvec;
+  void *q16, *k16;
+  int32_t *ord_r, *ord_c;
+  void *kg, *vg, *kg16;
+  float *dkg, *dvg;
+  size_t bytes;
+};
+
+BwdWs carve_bwd(void* base, int BH, int N, int d, int G) {
+  const size_t nb = (static_cast<size_t>(N) + kBlock - 1) / kBlock;
+  char* w = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = w == nullptr ? nullptr : w + off;
+    off += a256(bytes);
+    return p;
+  };
+  BwdWs r{};
+  r.lse2 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nb * kBlock * 4));
+  r.Dvec = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nb * kBlock * 4));
+  r.q16 = take(static_cast<size_t>(BH) * N * d * 2);
+  r.k16 = take(static_cast<size_t>(BH) * N * d * 2);
+  r.ord_r = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nb * 4));
+  r.ord_c = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nb * 4));
+  if (G > 0) {
+    const size_t gd = static_cast<size_t>(BH) * G * d;
+    r.kg = take(gd * 2);
+    r.vg = take(gd * 2);
+    r.kg16 = take(gd * 2);
+    r.dkg = reinterpret_cast<float*>(take(gd * 4));
+    r.dvg = reinterpret_cast<float*>(take(gd * 4));
+  }
+  r.bytes = off;
+  return r;
+}
 
 template <int D>
 cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
                            const int32_t* col_idx, const int32_t* col_ptr_t,
-                           const int32_t* row_idx_t, const int32_t* ord_r,
-                           const int32_t* ord_c, int BH, int N, float* lse2, float* Dvec,
-                           void* dq, void* dk, void* dv, unsigned int* err_word,
+                           const int32_t* row_idx_t, const BwdWs& ws, int BH, int N, int G,
+                           int gw, void* dq, void* dk, void* dv, unsigned int* err_word,
                            cudaStream_t stream) {
   using L = BwdLayout<D>;
   const int nb = (N + kBlock - 1) / kBlock;
   const int Np = nb * kBlock;
   const float c2 = kLog2e / sqrtf(static_cast<float>(D));
   const float scale = 1.f / sqrtf(static_cast<float>(D));
+  const float gbias2 = gw > 0 ? log2f(static_cast<float>(gw)) : 0.f;
   const long long limit = 1ll << 31;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(bwd_row_kernel<D, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
       (e = cudaFuncSetAttribute(bwd_row_kernel<D, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
-      (e = cudaFuncSetAttribute(bwd_col_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                L::kSmem)))
+      (e = cudaFuncSetAttribute(bwd_col_kernel<D, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
+      (e = cudaFuncSetAttribute(bwd_col_kernel<D, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)))
     return e;
+  static int regs_checked = 0;
+  if (regs_checked == 0) {
+    const void* fns[4] = {reinterpret_cast<const void*>(bwd_row_kernel<D, true>),
+                          reinterpret_cast<const void*>(bwd_row_kernel<D, false>),
+                          reinterpret_cast<const void*>(bwd_col_kernel<D, false>),
+                          reinterpret_cast<const void*>(bwd_col_kernel<D, true>)};
+    regs_checked = 1;
+    for (const void* fn : fns) {
+      cudaFuncAttributes fa{};
+      if ((e = cudaFuncGetAttributes(&fa, fn))) return e;
+      if (fa.numRegs != kLaunchRegs) regs_checked = -1;
+    }
+  }
+  if (regs_checked < 0) return cudaErrorInvalidConfiguration;
   const int grid = BH * nb;
-  // maps: Q16, dO, K16, V
+  // maps: Q16, dO, K16, V, Kg16, Vg (the last two stand in for K16, V without ASA_G)
   bwd_row_kernel<D, true><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], row_ptr, col_idx, ord_r, N, nb, Np, c2, scale, lse2,
-      Dvec, nullptr, err_word, limit);
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, ws.ord_r, N, nb,
+      Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, err_word, limit);
   if ((e = cudaGetLastError())) return e;
-  bwd_col_kernel<D><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[2], maps[3], maps[0], maps[1], col_ptr_t, row_idx_t, ord_c, N, nb, Np, c2, scale, lse2,
-      Dvec, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), err_word, limit);
+  if (G > 0) {
+    const int gtiles = BH * ((G + kBlock - 1) / kBlock);
+    bwd_col_kernel<D, true><<<gtiles, kBwdThreads, L::kSmem, stream>>>(
+        maps[4], maps[5], maps[0], maps[1], col_ptr_t, row_idx_t, ws.ord_c, N, nb, Np, G, gw,
+        gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, nullptr, ws.dkg, ws.dvg, err_word, limit);
+    if ((e = cudaGetLastError())) return e;
+  }
+  bwd_col_kernel<D, false><<<grid, kBwdThreads, L::kSmem, stream>>>(
+      maps[2], maps[3], maps[0], maps[1], col_ptr_t, row_idx_t, ws.ord_c, N, nb, Np, G, gw,
+      gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), ws.dkg, ws.dvg, err_word, limit);
   if ((e = cudaGetLastError())) return e;
   bwd_row_kernel<D, false><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], row_ptr, col_idx, ord_r, N, nb, Np, c2, scale, lse2,
-      Dvec, static_cast<__nv_bfloat16*>(dq), err_word, limit);
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, ws.ord_r, N, nb,
+      Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dq), err_word,
+      limit);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t bwd_tc_workspace_bytes(int BH, int N, int d) {
-  if (BH < 1 || N < 1) return 0;
-  const size_t nb = (static_cast<size_t>(N) + kBlock - 1) / kBlock;
-  const size_t vec = a256(static_cast<size_t>(BH) * nb * kBlock * sizeof(float));
-  const size_t cp = a256(static_cast<size_t>(BH) * N * d * 2);
-  const size_t ord = a256(static_cast<size_t>(BH) * nb * sizeof(int32_t));
-  return 2 * vec + 2 * cp + 2 * ord;
+size_t bwd_tc_workspace_bytes(int BH, int N, int d, int global_window) {
+  if (BH < 1 || N < 1 || global_window < 0) return 0;
+  const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
+  return carve_bwd(nullptr, BH, N, d, G).bytes;
 }
 
 cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const void* dout,
                           const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
-                          int d, void* workspace, void* dq, void* dk, void* dv,
+                          int d, int global_window, void* workspace, void* dq, void* dk, void* dv,
                           unsigned int* err_word, int num_sms, cudaStream_t stream) {
   const int nb = (N + kBlock - 1) / kBlock;
   const int Np = nb * kBlock;
-  char* w = static_cast<char*>(workspace);
-  const size_t vec = a256(static_cast<size_t>(BH) * Np * sizeof(float));
-  const size_t cp = a256(static_cast<size_t>(BH) * N * d * 2);
-  float* lse2 = reinterpret_cast<float*>(w);
-  float* Dvec = reinterpret_cast<float*>(w + vec);
-  void* q16 = w + 2 * vec;
-  void* k16 = w + 2 * vec + cp;
-  int32_t* ord_r = reinterpret_cast<int32_t*>(w + 2 * vec + 2 * cp);
-  int32_t* ord_c = ord_r + a256(static_cast<size_t>(BH) * nb * sizeof(int32_t)) / sizeof(int32_t);
+  const int gw = global_window;
+  const int G = gw > 0 ? (N + gw - 1) / gw : 0;
+  const BwdWs ws = carve_bwd(workspace, BH, N, d, G);
 
-  CUtensorMap maps[4];
-  if (!make_map_rows_f16(&maps[0], q16, BH, N, d) || !make_map_rows(&maps[1], dout, BH, N, d) ||
-      !make_map_rows_f16(&maps[2], k16, BH, N, d) || !make_map_rows(&maps[3], vp, BH, N, d))
+  CUtensorMap maps[6];
+  if (!make_map_rows_f16(&maps[0], ws.q16, BH, N, d) ||
+      !make_map_rows(&maps[1], dout, BH, N, d) ||
+      !make_map_rows_f16(&maps[2], ws.k16, BH, N, d) || !make_map_rows(&maps[3], vp, BH, N, d))
     return cudaErrorInvalidValue;
+  if (G > 0) {
+    if (!make_map_rows_f16(&maps[4], ws.kg16, BH, G, d) ||
+        !make_map_rows(&maps[5], ws.vg, BH, G, d))
+      return cudaErrorInvalidValue;
+  } else {
+    maps[4] = maps[2];
+    maps[5] = maps[3];
+  }
 
-  const int64_t n8 = static_cast<int64_t>(BH) * N * d / 8;
   const int blocks = num_sms * 8;
   bwd_prep_kernel<<<blocks, 256, 0, stream>>>(
-      static_cast<const uint4*>(qp), static_cast<const uint4*>(kp), static_cast<uint4*>(q16),
-      static_cast<uint4*>(k16), n8, lse, lse2, Dvec, BH, N, Np, err_word);
+      static_cast<const uint4*>(qp), static_cast<const uint4*>(kp), static_cast<uint4*>(ws.q16),
+      static_cast<uint4*>(ws.k16), static_cast<int64_t>(BH) * N * d / 8, lse, ws.lse2, ws.Dvec,
+      BH, N, Np, err_word);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, ord_r, stream);
-  if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, ord_c, stream);
+  if (e == cudaSuccess && G > 0) {
+    // the forward's global tokens, recomputed: mean-pooled K and V, Kg also in fp16
+    e = launch_global_pool(kp, ws.kg, BH, N, d, gw, num_sms, stream);
+    if (e == cudaSuccess) e = launch_global_pool(vp, ws.vg, BH, N, d, gw, num_sms, stream);
+    if (e == cudaSuccess) {
+      f16_copy_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(ws.kg),
+                                                  static_cast<uint4*>(ws.kg16),
+                                                  static_cast<int64_t>(BH) * G * d / 8, err_word);
+      e = cudaGetLastError();
+    }
+  }
+  if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, ws.ord_r, stream);
+  if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, ws.ord_c, stream);
   if (e != cudaSuccess) return e;
   if (d == 128)
-    return launch_kernels<128>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ord_r, ord_c, BH, N,
-                               lse2, Dvec, dq, dk, dv, err_word, stream);
-  return launch_kernels<64>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ord_r, ord_c, BH, N,
-                            lse2, Dvec, dq, dk, dv, err_word, stream);
+    return launch_kernels<128>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ws, BH, N, G, gw,
+                               dq, dk, dv, err_word, stream);
+  return launch_kernels<64>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ws, BH, N, G, gw, dq,
+                            dk, dv, err_word, stream);
 }
 
 }  // namespace asa

@@ -47,12 +47,13 @@ cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
                              cudaStream_t stream);
 
 // Backward workspace (bytes, 256-aligned pieces): lse2 and D [BH][nb*128] f32,
-// fp16 copies of Q and K [BH][N][d], launch orders of query and key blocks [BH*nb].
-size_t bwd_tc_workspace_bytes(int BH, int N, int d);
+// fp16 copies of Q and K [BH][N][d], launch orders of query and key blocks [BH*nb];
+// with ASA_G the global tokens and their fp32 gradients.
+size_t bwd_tc_workspace_bytes(int BH, int N, int d, int global_window);
 cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const void* dout,
                           const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
-                          int d, void* workspace, void* dq, void* dk, void* dv,
-                          unsigned int* err_word, int num_sms, cudaStream_t stream);
+                          int d, int global_window, void* workspace, void* dq, void* dk,
+                          void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream);
 
 }  // namespace asa
