@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "wan2.1-1.3b"
 METRIC = "ASA ms/call & effective TFLOP/s at 32760 tok, H=12, d=128, τ=0.95"
-KERNELS_PER_STEP = 9   # permute3, est_logits, est_pool, mask_rows, scan, fill, lpt_order, fwd, unpermute
+KERNELS_PER_STEP = 11  # permute3, est_gather, est_tc, est_combine, est_pool, mask_rows, scan, fill, lpt_order, fwd, unpermute
 
 
 def _peaks():
@@ -281,8 +281,9 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
     asa.asa_gilbert_permute3(q, k, v, T, Hg, W, outs=(qp, kp, vp))
     ws = asa.estimate_mask_workspace(B, H, N, dev)
     p_imp = torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
-    mask = asa._alloc_mask(B, H, N, dev, transposed=wl.backward)
     gw = wl.global_window
+    want_bwd = wl.backward or gw > 0
+    mask = asa._alloc_mask(B, H, N, dev, transposed=want_bwd)
     fws = asa.fwd_workspace(B, H, N, d, gw, dev)
     op = torch.empty_like(qp)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -301,9 +302,9 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
     hbm_stage("permute_qkv", lambda: asa.asa_gilbert_permute3(q, k, v, T, Hg, W, outs=(qp, kp, vp)),
               3 * 2 * tensor_bytes)
     r["estimate"] = timer(lambda: asa.asa_estimate(qp, kp, workspace=ws, out=p_imp))
-    r["mask"] = timer(lambda: asa.asa_build_mask(p_imp, N, wl.tau, transposed=wl.backward,
+    r["mask"] = timer(lambda: asa.asa_build_mask(p_imp, N, wl.tau, transposed=want_bwd,
                                                  workspace=ws, mask=mask))
-    r["estimate_mask"] = timer(lambda: asa.asa_estimate_mask(qp, kp, wl.tau, transposed=wl.backward,
+    r["estimate_mask"] = timer(lambda: asa.asa_estimate_mask(qp, kp, wl.tau, transposed=want_bwd,
                                                              workspace=ws, mask=mask))
     torch.cuda.synchronize()
     Ls = np.array([min(128, N - 128 * i) for i in range(nb)])
@@ -332,13 +333,16 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
     hbm_stage("unpermute_o", lambda: asa.asa_unpermute(op, T, Hg, W, out=out), 2 * tensor_bytes)
     em = r["estimate_mask"]["median_ms"]
     r["estimate_mask_share"] = em / (em + r["attn_fwd"]["median_ms"])
-    if wl.backward:
-        do = x["dout"].to(dev)
-        dop = asa.asa_gilbert_permute(do, T, Hg, W)
-        bws = asa.bwd_workspace(B, H, N, d, dev)
+    if want_bwd:
+        if wl.backward:
+            dop = asa.asa_gilbert_permute(x["dout"].to(dev), T, Hg, W)
+        else:
+            dop = torch.randn_like(qp)
+        bws = asa.bwd_workspace(B, H, N, d, dev, gw)
         grads = tuple(torch.empty_like(qp) for _ in range(3))
         r["attn_bwd"] = timer(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, mask,
-                                                              workspace=bws, outs=grads),
+                                                              global_window=gw, workspace=bws,
+                                                              outs=grads),
                               reps=8, warm=3)
         tb = r["attn_bwd"]["median_ms"] * 1e-3
         r["attn_bwd"]["effective_TFLOP_s"] = 2.5 * flops / tb / 1e12
@@ -610,6 +614,10 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
     bwd_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, tmask), reps=5)
     flops, _, _ = _kept_tile_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
                                    B, H, N, d)
+    # ASA_G backward (n = 64) on the same mask
+    og, lg = asa.asa_sparse_attn_fwd(qp, kp, vp, tmask, global_window=64)
+    bwd_g_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, og, dout, lg, tmask,
+                                                      global_window=64), reps=5)
     G = -(-N // 64)
     return {
         "dense_ours_fwd_ms": ours_dense, "dense_ours_tflops": dense_flops / ours_dense / 1e9,
@@ -617,6 +625,8 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
         "asa_g_fwd_ms_n64": g_ms,
         "asa_g_fwd_tflops": (flops + 4 * d * N * G * B * H) / g_ms / 1e9,
         "bwd_ms": bwd_ms, "bwd_tflops": 2.5 * flops / bwd_ms / 1e9,
+        "asa_g_bwd_ms_n64": bwd_g_ms,
+        "asa_g_bwd_tflops": 2.5 * (flops + 4 * d * N * G * B * H) / bwd_g_ms / 1e9,
     }
 
 
