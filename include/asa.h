@@ -224,6 +224,16 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
  */
 int asa_check_device_status(void* stream);
 
+/*
+ * Test hook for failure detection (no counterpart on the pages): launches one CTA whose
+ * bounded mbarrier wait (the primitive every kernel uses) waits on a barrier that
+ * nothing ever arrives at, so it gives up after `limit_cycles` SM clock cycles (1 to
+ * 2^31, about 1 s at most), records the expiry in the device error word and returns.
+ * The next asa_check_device_status then returns ASA_ERR_TIMEOUT and clears the word;
+ * the context stays usable.  Asynchronous on `stream`; nothing else calls it.
+ */
+int asa_selftest_wait_timeout(long long limit_cycles, void* stream);
+
 /* Frees the cached permutation tables of every device.  Safe to call twice. */
 void asa_shutdown(void);
 

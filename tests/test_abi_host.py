@@ -129,6 +129,12 @@ def test_attention_rejects(L):
     assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_INVALID_ARG
 
 
+def test_selftest_rejects_bad_limits(L):
+    assert L.asa_selftest_wait_timeout(0, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_selftest_wait_timeout((1 << 31) + 1, None) == asa.ASA_ERR_INVALID_ARG
+    assert b"limit_cycles" in L.asa_last_error_string()
+
+
 def test_workspace_sizes(L):
     nb = 256
     est = L.asa_estimate_mask_workspace_size(1, 12, 32760)

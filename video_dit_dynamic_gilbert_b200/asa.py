@@ -44,6 +44,7 @@ _SIGNATURES = {
     "asa_bwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_check_device_status": ([_vp], _c_int),
+    "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),
 }
 
@@ -297,6 +298,11 @@ def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, global_window
 
 def asa_check_device_status(stream=None) -> None:
     _check(lib().asa_check_device_status(_stream(stream)))
+
+
+def asa_selftest_wait_timeout(limit_cycles: int = 1 << 20, stream=None) -> None:
+    """Failure-detection test hook: one bounded wait that must give up (see asa.h)."""
+    _check(lib().asa_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
 
 
 def asa_shutdown() -> None:

@@ -432,6 +432,17 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
   return ASA_OK;
 }
 
+int asa_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > (1ll << 31))
+    return fail(ASA_ERR_INVALID_ARG, "limit_cycles=%lld outside [1, 2^31]", limit_cycles);
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_wait_timeout(err_word, limit_cycles, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ASA_OK;
+}
+
 int asa_check_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

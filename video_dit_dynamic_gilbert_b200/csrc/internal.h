@@ -56,4 +56,7 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           int d, int global_window, void* workspace, void* dq, void* dk,
                           void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream);
 
+// Failure-detection test hook: one bounded wait on a barrier nothing arrives at.
+cudaError_t launch_wait_timeout(unsigned int* err_word, long long limit, cudaStream_t stream);
+
 }  // namespace asa
