@@ -319,3 +319,38 @@ def asa_attention(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: i
     mask = asa_estimate_mask(qp, kp, tau, transposed=False, stream=stream)
     op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window, stream=stream)
     return asa_unpermute(op, T, Hg, W, stream=stream), lse, mask
+
+
+class ASAAttention(torch.autograd.Function):
+    """ASA (or ASA_G) self-attention as a differentiable op on raster-layout q, k, v
+    [B, N, H, d] bf16.  The mask is computed in the forward from q and k and is not
+    differentiated (the pages fix it for training as for inference); the backward is
+    asa_sparse_attn_bwd under that mask, its gradients unpermuted to raster layout."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0):
+        q, k, v = (t.contiguous() for t in (q, k, v))
+        qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W)
+        mask = asa_estimate_mask(qp, kp, tau, transposed=True)
+        op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window)
+        ctx.save_for_backward(qp, kp, vp, op, lse)
+        ctx.mask, ctx.grid, ctx.global_window = mask, (T, Hg, W), global_window
+        return asa_unpermute(op, T, Hg, W)
+
+    @staticmethod
+    def backward(ctx, dout):
+        qp, kp, vp, op, lse = ctx.saved_tensors
+        T, Hg, W = ctx.grid
+        dop = asa_gilbert_permute(dout.to(torch.bfloat16).contiguous(), T, Hg, W)
+        grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
+                                    global_window=ctx.global_window)
+        dq, dk, dv = (asa_unpermute(g, T, Hg, W) for g in grads)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def asa_attention_trainable(q, k, v, T: int, Hg: int, W: int, tau: float,
+                            global_window: int = 0):
+    """Differentiable asa_attention: returns O [B, N, H, d] (raster); gradients flow to
+    q, k and v through the kernels' backward under the forward's mask."""
+    return ASAAttention.apply(q, k, v, T, Hg, W, tau, global_window)
+
