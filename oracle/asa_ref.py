@@ -93,28 +93,35 @@ def unpermute(xp: np.ndarray, perm: np.ndarray) -> np.ndarray:
 # Step 1: block importance estimation
 # ----------------------------------------------------------------------------
 
-def estimate_pimp(qp: np.ndarray, kp: np.ndarray, b: int = 128, k: int = 16) -> np.ndarray:
+def estimate_pimp(qp: np.ndarray, kp: np.ndarray, b: int = 128, k: int = 16,
+                  q_blocks=None) -> np.ndarray:
     """P_imp [B, H, nb, nb] from k sampled tokens per block.
 
     Q_s, K_s = sampled rows; P_approx = softmax(Q_s K_s^T / sqrt(d)) over each row;
     P_imp[I, J] = max of the (rows of block I) x (columns of block J) tile.
     With k >= b every token is sampled and this is the exact max-pool of the full
     attention map that the section describes first.
+    q_blocks: compute only these rows of P_imp (each row needs only its own block's
+    sample rows against every sampled key); returns [B, H, len(q_blocks), nb].
     """
     B, H, N, d = qp.shape
     rows = sample_rows(N, b, k)
     starts = _sample_block_starts(N, b, k)
     nb = len(starts)
-    out = np.empty((B, H, nb, nb), dtype=np.float64)
+    sel = np.arange(nb) if q_blocks is None else np.asarray(list(q_blocks), dtype=np.int64)
+    ends = np.append(starts[1:], len(rows))
+    qrows = np.concatenate([np.arange(starts[I], ends[I]) for I in sel])
+    qstarts = np.concatenate([[0], np.cumsum(ends[sel] - starts[sel])[:-1]]).astype(np.int64)
+    out = np.empty((B, H, len(sel), nb), dtype=np.float64)
     for bb in range(B):
         for h in range(H):
-            Qs = np.asarray(qp[bb, h, rows, :], dtype=np.float64)
+            Qs = np.asarray(qp[bb, h, rows[qrows], :], dtype=np.float64)
             Ks = np.asarray(kp[bb, h, rows, :], dtype=np.float64)
             S = (Qs @ Ks.T) / math.sqrt(d)
             S = S - S.max(axis=1, keepdims=True)
             P = np.exp(S)
             P = P / P.sum(axis=1, keepdims=True)
-            tile_max = np.maximum.reduceat(np.maximum.reduceat(P, starts, axis=0), starts, axis=1)
+            tile_max = np.maximum.reduceat(np.maximum.reduceat(P, qstarts, axis=0), starts, axis=1)
             out[bb, h] = tile_max
     return out
 

@@ -170,3 +170,17 @@ def test_csr_round_trip():
             r = bh * 5 + J
             rows = ti[tp[r]:tp[r + 1]]
             assert rows.tolist() == np.nonzero(mask.reshape(6, 5, 5)[bh, :, J])[0].tolist()
+
+
+def test_estimate_pimp_block_selection_matches_full():
+    """Selecting query blocks only picks rows: each P_imp row needs only its own block's
+    sample rows (ragged last block and a block shorter than k included)."""
+    g = np.random.default_rng(17)
+    N, d = 128 * 5 + 9, 16
+    q = g.standard_normal((2, 2, N, d))
+    k = g.standard_normal((2, 2, N, d))
+    full = oracle.estimate_pimp(q, k)
+    sel = [4, 0, 5, 2]
+    part = oracle.estimate_pimp(q, k, q_blocks=sel)
+    assert part.shape == (2, 2, len(sel), full.shape[-1])
+    np.testing.assert_allclose(part, full[:, :, sel], rtol=1e-13, atol=1e-15)

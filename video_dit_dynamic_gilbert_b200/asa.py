@@ -92,6 +92,10 @@ def _bf16_cuda(name: str, t: torch.Tensor, ndim: int = 4) -> None:
         raise ValueError(f"{name} must be a contiguous {ndim}-D bf16 CUDA tensor")
 
 
+def _ws_bytes(workspace) -> int:
+    return 0 if workspace is None else workspace.numel()
+
+
 def _workspace(nbytes: int, device) -> torch.Tensor | None:
     if nbytes == 0:
         return None
@@ -186,7 +190,7 @@ def asa_estimate(qp: torch.Tensor, kp: torch.Tensor, workspace=None, out=None, s
     if out is None:
         out = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qp.device)
     _check(lib().asa_estimate(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, _ptr(workspace),
-                              workspace.numel(), _ptr(out), _stream(stream)))
+                              _ws_bytes(workspace), _ptr(out), _stream(stream)))
     return out
 
 
@@ -214,7 +218,7 @@ def asa_build_mask(p_imp: torch.Tensor, N: int, tau: float, transposed: bool = T
     if workspace is None:
         workspace = estimate_mask_workspace(B, H, N, p_imp.device)
     m = mask or _alloc_mask(B, H, N, p_imp.device, transposed)
-    _check(lib().asa_build_mask(_ptr(p_imp), B, H, N, float(tau), _ptr(workspace), workspace.numel(),
+    _check(lib().asa_build_mask(_ptr(p_imp), B, H, N, float(tau), _ptr(workspace), _ws_bytes(workspace),
                                 _ptr(m.row_ptr), _ptr(m.col_idx), _ptr(m.nnz), _ptr(m.col_ptr_t),
                                 _ptr(m.row_idx_t), _stream(stream)))
     return m
@@ -230,7 +234,7 @@ def asa_estimate_mask(qp: torch.Tensor, kp: torch.Tensor, tau: float, transposed
         workspace = estimate_mask_workspace(B, H, N, qp.device)
     m = mask or _alloc_mask(B, H, N, qp.device, transposed)
     _check(lib().asa_estimate_mask(_ptr(qp), _ptr(kp), B, H, N, d, BLOCK, SAMPLES, float(tau),
-                                   _ptr(workspace), workspace.numel(), _ptr(m.row_ptr),
+                                   _ptr(workspace), _ws_bytes(workspace), _ptr(m.row_ptr),
                                    _ptr(m.col_idx), _ptr(m.nnz), _ptr(m.col_ptr_t),
                                    _ptr(m.row_idx_t), _stream(stream)))
     return m
@@ -266,7 +270,7 @@ def asa_sparse_attn_fwd(qp, kp, vp, mask: BlockMask, global_window: int = 0, wor
         lse = torch.empty((B, H, N), dtype=torch.float32, device=qp.device)
     _check(lib().asa_sparse_attn_fwd(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(mask.row_ptr),
                                      _ptr(mask.col_idx), B, H, N, d, BLOCK, global_window,
-                                     _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                     _ptr(workspace), _ws_bytes(workspace),
                                      _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
@@ -292,7 +296,7 @@ def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, global_window
                                      _ptr(mask.row_ptr), _ptr(mask.col_idx), _ptr(mask.col_ptr_t),
                                      _ptr(mask.row_idx_t), B, H, N, d, BLOCK, global_window,
                                      _ptr(workspace),
-                                     workspace.numel(), *(_ptr(t) for t in outs), _stream(stream)))
+                                     _ws_bytes(workspace), *(_ptr(t) for t in outs), _stream(stream)))
     return outs
 
 
