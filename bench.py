@@ -312,6 +312,14 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
     est_flops = 2 * M * M * d * B * H
     r["estimate"]["TFLOP_s"] = est_flops / (r["estimate"]["median_ms"] * 1e-3) / 1e12
     r["estimate"]["exp_count"] = M * M * B * H
+    # the second mask mode (statistical threshold), about a quarter of the blocks per row
+    mstat = asa._alloc_mask(B, H, N, dev, transposed=False)
+    r["mask_stat"] = timer(lambda: asa.asa_build_mask_stat(p_imp, N, max(1, nb // 4),
+                                                           transposed=False, workspace=ws,
+                                                           mask=mstat))
+    torch.cuda.synchronize()
+    r["mask_stat"]["k_target"] = max(1, nb // 4)
+    r["mask_stat"]["kept_fraction"] = int(mstat.nnz.item()) / (B * H * nb * nb)
     near, rows = _near_threshold_rows(p_imp.cpu().numpy(), wl.tau)
     r["near_threshold_rows"] = {"count": near, "of": rows}
     flops, nnz, tiles = _kept_tile_flops(mask.row_ptr.cpu().numpy(), mask.col_idx.cpu().numpy(),

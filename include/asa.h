@@ -146,6 +146,22 @@ int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* wor
 int asa_estimate_noalloc(const void* qp, const void* kp, int B, int H, int N, int d, int block,
                          int samples, float* p_imp, void* stream);
 
+/*
+ * Statistical-threshold mask, a second mask mode with the same inputs and outputs as
+ * asa_build_mask: BSA's adaptive key-block selection (the BSA page, design point 2:
+ * p = mean(S_b) + std(S_b) * U(1 - k/n), U the normal quantile function, n the number
+ * of blocks, k the target candidate count).  Reading
+ * taken: per query block, S_b are the row's shares R_J = P_imp[I, J] / sum_J P_imp[I, J];
+ * p = mean(R) + std(R) * Phi^-1(1 - k_target/nb) (population std); every key block with
+ * R_J >= p is kept (about k_target of nb blocks when the shares are normal); a row that
+ * keeps none keeps its largest share (lowest J on ties).  k_target >= nb keeps every
+ * block.  Sums in fp64.  p_imp: device fp32 [B, H, nb, nb]; the workspace and the CSR
+ * outputs are those of asa_build_mask.
+ */
+int asa_build_mask_stat(const float* p_imp, int B, int H, int N, int k_target, void* workspace,
+                        size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                        int32_t* col_ptr_t, int32_t* row_idx_t, void* stream);
+
 /* Steps 1 + 2.1 in one call (P_imp stays in the workspace). Arguments as above. */
 int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d, int block,
                       int samples, float tau, void* workspace, size_t ws_bytes, int32_t* row_ptr,

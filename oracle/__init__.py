@@ -29,6 +29,9 @@ Parity status per function (how each is pinned is in tests/test_oracle_*.py):
                      additive ln(n) mask; n=1 closed form.
   asa_backward       pinned: torch.autograd of masked SDPA fp64; central finite
                      differences on a tiny case.
+  build_mask_stat    pinned: k = n/2 keeps exactly the shares >= 1/n (U(1/2) = 0);
+                     normal-distributed shares keep about k of n blocks (a flipped
+                     quantile keeps n - k); the all-below fallback; k >= n keeps all.
 """
 from .gilbert import gilbert_order  # noqa: F401
 from .asa_ref import (  # noqa: F401
@@ -39,6 +42,8 @@ from .asa_ref import (  # noqa: F401
     unpermute,
     estimate_pimp,
     build_mask,
+    build_mask_stat,
+    marginal_rows_stat,
     mask_to_csr,
     mask_to_csr_transposed,
     marginal_rows,

@@ -30,7 +30,10 @@ Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
   * LSE is the natural-log log-sum-exp of the logits a query row attends to;
   * in the ASA_G backward the gradient of a global token reaches the rows of its
     window through the mean (divided by the window's row count); its bf16 rounding
-    passes gradients unchanged.
+    passes gradients unchanged;
+  * the statistical threshold (BSA page) is a threshold on each block's share, not a
+    cumulative target: with U(1 - k/n) the normal quantile it keeps about k of n blocks;
+    a row that keeps none keeps its largest share.
 """
 from __future__ import annotations
 
@@ -156,6 +159,64 @@ def build_mask(pimp: np.ndarray, tau: float) -> np.ndarray:
                 c = _row_cut(share, order, tau)
                 mask[bb, h, I, order[:c]] = True
     return mask
+
+
+def build_mask_stat(pimp: np.ndarray, k_target: int) -> np.ndarray:
+    """Statistical-threshold mask [B, H, rows, nb] (BSA's adaptive KV selection,
+    p = mean(S_b) + std(S_b) U(1 - k/n), U the standard normal quantile function).
+
+    Per row: shares R = P_imp / sum(P_imp); p = mean(R) + std(R) * U(1 - k/n) with n the
+    number of key blocks and the population std; keep every block with R >= p; a row
+    that keeps none keeps its largest share (lowest J on ties); k >= n keeps all.
+    """
+    from scipy.stats import norm
+    B, H, nr, nb = pimp.shape
+    mask = np.zeros(pimp.shape, dtype=bool)
+    if k_target >= nb:
+        mask[:] = True
+        return mask
+    z = norm.ppf(1.0 - k_target / nb)
+    for bb in range(B):
+        for h in range(H):
+            for I in range(nr):
+                v = np.maximum(np.asarray(pimp[bb, h, I], dtype=np.float64), 0.0)
+                total = v.sum()
+                if not total > 0:
+                    mask[bb, h, I] = True
+                    continue
+                R = v / total
+                p = R.mean() + R.std() * z
+                keep = R >= p
+                if not keep.any():
+                    keep[int(np.argmax(R))] = True
+                mask[bb, h, I] = keep
+    return mask
+
+
+def marginal_rows_stat(pimp: np.ndarray, k_target: int, eps: float = 1e-9) -> np.ndarray:
+    """Rows whose statistical-threshold decision an fp32 evaluation may place
+    differently: some share within ``eps`` (relative) of the threshold, or a fallback row
+    whose largest shares tie within ``eps``."""
+    from scipy.stats import norm
+    B, H, nr, nb = pimp.shape
+    marg = np.zeros((B, H, nr), dtype=bool)
+    if k_target >= nb:
+        return marg
+    z = norm.ppf(1.0 - k_target / nb)
+    for bb in range(B):
+        for h in range(H):
+            for I in range(nr):
+                v = np.maximum(np.asarray(pimp[bb, h, I], dtype=np.float64), 0.0)
+                if not v.sum() > 0:
+                    continue
+                R = v / v.sum()
+                p = R.mean() + R.std() * z
+                m = np.abs(R - p).min() <= eps * max(abs(p), 1e-300)
+                if not (R >= p).any():
+                    top = np.sort(R)[::-1]
+                    m |= len(top) > 1 and top[0] - top[1] <= eps * top[0]
+                marg[bb, h, I] = m
+    return marg
 
 
 def marginal_rows(pimp: np.ndarray, tau: float, eps: float = 1e-4,

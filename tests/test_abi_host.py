@@ -129,6 +129,16 @@ def test_attention_rejects(L):
     assert L.asa_sparse_attn_bwd(*args) == asa.ASA_ERR_INVALID_ARG
 
 
+def test_stat_mask_rejects(L):
+    args = lambda k=4, ws=None, wsb=0: (FAKE, 1, 2, 1024, k, ws, wsb, FAKE, FAKE, FAKE, None, None,
+                                        None)
+    assert L.asa_build_mask_stat(*args(k=0)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_build_mask_stat(*args()) == asa.ASA_ERR_WORKSPACE
+    bad = list(args(ws=ctypes.c_void_p(0x100000), wsb=1 << 30))
+    bad[10] = FAKE          # col_ptr_t without row_idx_t
+    assert L.asa_build_mask_stat(*bad) == asa.ASA_ERR_INVALID_ARG
+
+
 def test_selftest_rejects_bad_limits(L):
     assert L.asa_selftest_wait_timeout(0, None) == asa.ASA_ERR_INVALID_ARG
     assert L.asa_selftest_wait_timeout((1 << 31) + 1, None) == asa.ASA_ERR_INVALID_ARG

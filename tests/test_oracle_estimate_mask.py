@@ -184,3 +184,45 @@ def test_estimate_pimp_block_selection_matches_full():
     part = oracle.estimate_pimp(q, k, q_blocks=sel)
     assert part.shape == (2, 2, len(sel), full.shape[-1])
     np.testing.assert_allclose(part, full[:, :, sel], rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- statistical threshold
+
+def test_stat_mask_median_quantile_keeps_shares_above_mean():
+    """k = n/2: U(1/2) = 0, so the threshold is the mean share 1/n exactly."""
+    row = np.array([5.0, 1.0, 1.0, 3.0, 0.5, 2.0, 2.5, 1.0])   # mean 2.0 -> shares >= 1/8
+    m = oracle.build_mask_stat(row[None, None, None, :], 4)
+    assert m[0, 0, 0].tolist() == [True, False, False, True, False, True, True, False]
+
+
+def test_stat_mask_keeps_about_k_of_n_for_normal_shares():
+    """Shares drawn from a normal distribution: about k of n blocks lie above
+    mean + std U(1 - k/n).  A flipped quantile (U(k/n)) would keep n - k."""
+    g = np.random.default_rng(5)
+    n, k, rows = 2000, 200, 40
+    p = 10.0 + g.standard_normal((1, 1, rows, n))
+    kept = oracle.build_mask_stat(p, k).sum(-1)
+    assert abs(kept.mean() - k) < 15
+    assert kept.min() > 140 and kept.max() < 260
+
+
+def test_stat_mask_fallback_and_keep_all():
+    # every share equal except one slightly lower: the threshold sits above the equal
+    # ones, so none passes and the largest share (lowest J) is kept
+    row = np.full(1000, 1.0)
+    row[7] = 0.9
+    m = oracle.build_mask_stat(row[None, None, None, :], 1)
+    assert m.sum() == 1 and m[0, 0, 0, 0]
+    assert oracle.build_mask_stat(row[None, None, None, :], 1000).all()
+    assert oracle.build_mask_stat(row[None, None, None, :], 5000).all()
+
+
+def test_stat_mask_quantile_matches_table_values():
+    """The threshold uses the standard normal quantile: U(0.75) = 0.674490 (table)."""
+    n, k = 40, 10                     # 1 - k/n = 0.75
+    R = np.linspace(1.0, 2.0, n)
+    m = oracle.build_mask_stat(R[None, None, None, :], k)
+    s = R / R.sum()
+    want = s >= s.mean() + s.std() * 0.674490
+    assert 0 < want.sum() < n
+    assert m[0, 0, 0].tolist() == want.tolist()

@@ -43,6 +43,7 @@ _SIGNATURES = {
     "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
     "asa_bwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
+    "asa_build_mask_stat": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size] + [_vp] * 6, _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),
@@ -221,6 +222,22 @@ def asa_build_mask(p_imp: torch.Tensor, N: int, tau: float, transposed: bool = T
     _check(lib().asa_build_mask(_ptr(p_imp), B, H, N, float(tau), _ptr(workspace), _ws_bytes(workspace),
                                 _ptr(m.row_ptr), _ptr(m.col_idx), _ptr(m.nnz), _ptr(m.col_ptr_t),
                                 _ptr(m.row_idx_t), _stream(stream)))
+    return m
+
+
+def asa_build_mask_stat(p_imp: torch.Tensor, N: int, k_target: int, transposed: bool = True,
+                        workspace=None, mask: BlockMask | None = None, stream=None) -> BlockMask:
+    """Kept-block CSR by the statistical threshold (about k_target blocks per row)."""
+    if not (p_imp.is_cuda and p_imp.dtype == torch.float32 and p_imp.is_contiguous()):
+        raise ValueError("p_imp must be a contiguous fp32 CUDA tensor")
+    B, H = p_imp.shape[:2]
+    if workspace is None:
+        workspace = estimate_mask_workspace(B, H, N, p_imp.device)
+    m = mask or _alloc_mask(B, H, N, p_imp.device, transposed)
+    _check(lib().asa_build_mask_stat(_ptr(p_imp), B, H, N, int(k_target), _ptr(workspace),
+                                     _ws_bytes(workspace), _ptr(m.row_ptr), _ptr(m.col_idx),
+                                     _ptr(m.nnz), _ptr(m.col_ptr_t), _ptr(m.row_idx_t),
+                                     _stream(stream)))
     return m
 
 

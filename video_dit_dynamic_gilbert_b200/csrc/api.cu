@@ -312,6 +312,37 @@ int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* wor
                          stream);
 }
 
+// Phi^-1(p) for 0 < p < 1: bisection on the standard normal CDF 0.5 erfc(-x / sqrt 2),
+// to the resolution of double
+static double normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 200 && hi - lo > 1e-15 * (1.0 + std::fabs(lo)); ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+int asa_build_mask_stat(const float* p_imp, int B, int H, int N, int k_target, void* workspace,
+                        size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                        int32_t* col_ptr_t, int32_t* row_idx_t, void* stream) {
+  ASA_TRY(check_common(B, H, N, 64));
+  ASA_TRY(check_ptr(p_imp, "p_imp", false));
+  if (k_target < 1) return fail(ASA_ERR_INVALID_ARG, "k_target=%d must be >= 1", k_target);
+  ASA_TRY(check_mask_args(1.f, row_ptr, col_idx, nnz_out, col_ptr_t, row_idx_t));
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  MaskWs w = carve_mask_ws(workspace, B * H, nb);
+  ASA_TRY(check_ws(workspace, ws_bytes, w.bytes));
+  const bool keep_all = k_target >= nb;
+  const double z = keep_all ? 0.0 : normal_quantile(1.0 - static_cast<double>(k_target) / nb);
+  cudaError_t e = asa::launch_build_mask_stat(p_imp, B * H, nb, z, keep_all, w.bitmap, w.counts,
+                                              row_ptr, col_idx, nnz_out, w.counts_t, col_ptr_t,
+                                              row_idx_t, num_sms_current(),
+                                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
+  return ASA_OK;
+}
+
 int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d, int block,
                       int samples, float tau, void* workspace, size_t ws_bytes, int32_t* row_ptr,
                       int32_t* col_idx, int32_t* nnz_out, int32_t* col_ptr_t, int32_t* row_idx_t,

@@ -33,6 +33,13 @@ cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uin
                               int32_t* counts_t, int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,
                               cudaStream_t stream);
 
+// Statistical-threshold mask: z = Phi^-1(1 - k/n); keep_all when k >= n.
+cudaError_t launch_build_mask_stat(const float* p_imp, int BH, int nb, double z, bool keep_all,
+                                   uint8_t* bitmap, int32_t* counts, int32_t* row_ptr,
+                                   int32_t* col_idx, int32_t* nnz_out, int32_t* counts_t,
+                                   int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,
+                                   cudaStream_t stream);
+
 cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, int n, int num_sms,
                                cudaStream_t stream);
 

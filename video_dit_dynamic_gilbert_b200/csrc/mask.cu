@@ -10,7 +10,12 @@
 // the row.  Blocks above v* are kept, and blocks equal to v* are added in J order
 // until the cumulative sum reaches the target.  Sums are taken in fp64.
 //
-// Kernels: mask_rows (one warp per row) -> bitmap [rows][nb] + counts; scan ->
+// Statistical threshold (the BSA mode; "Video-BLADE" names BSA's adaptive selection as
+// related work): shares R as above, p = mean(R) + std(R) z with z = Phi^-1(1 - k/n)
+// (computed on the host), keep every block with R >= p; a row that keeps none keeps its
+// largest share (lowest J on ties).  Sums in fp64.
+//
+// Kernels: mask_rows / stat_rows (one warp per row) -> bitmap [rows][nb] + counts; scan ->
 // row_ptr (+ nnz); fill -> col_idx (J ascending); and for the transposed CSR
 // (per key block the query blocks that keep it): tcount -> scan -> tfill.
 #include "common.cuh"
@@ -82,6 +87,63 @@ __global__ void __launch_bounds__(kMaskWarps * 32)
       if (J < nb) brow[J] = keep ? 1 : 0;
       kept += __popc(__ballot_sync(0xffffffffu, keep));
       ties_seen += __popc(tmask);
+    }
+    if (lane == 0) counts[row] = kept;
+  }
+}
+
+// Statistical threshold, one warp per row; keep_all: k >= nb (every block)
+__global__ void __launch_bounds__(kMaskWarps * 32)
+    stat_rows_kernel(const float* __restrict__ p_imp, int rows, int nb, double z, int keep_all,
+                     uint8_t* __restrict__ bitmap, int32_t* __restrict__ counts) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int row = blockIdx.x * kMaskWarps + warp; row < rows; row += gridDim.x * kMaskWarps) {
+    const float* src = p_imp + static_cast<int64_t>(row) * nb;
+    uint8_t* brow = bitmap + static_cast<int64_t>(row) * nb;
+    double part = 0.0;
+    for (int J = lane; J < nb; J += 32) part += fmaxf(src[J], 0.f);
+    const double total = warp_sum_d(part);
+    if (keep_all || !(total > 0.0)) {
+      for (int J = lane; J < nb; J += 32) brow[J] = 1;
+      if (lane == 0) counts[row] = nb;
+      continue;
+    }
+    double sr = 0.0;
+    for (int J = lane; J < nb; J += 32) sr += fmaxf(src[J], 0.f) / total;
+    const double mean = warp_sum_d(sr) / nb;
+    double sq = 0.0;
+    for (int J = lane; J < nb; J += 32) {
+      const double dv = fmaxf(src[J], 0.f) / total - mean;
+      sq += dv * dv;
+    }
+    const double thr = mean + sqrt(warp_sum_d(sq) / nb) * z;
+    int kept = 0;
+    float best = -1.f;
+    int best_j = nb;
+    for (int J0 = 0; J0 < nb; J0 += 32) {
+      const int J = J0 + lane;
+      const float v = J < nb ? fmaxf(src[J], 0.f) : -1.f;
+      const bool keep = J < nb && static_cast<double>(v) / total >= thr;
+      if (J < nb) brow[J] = keep ? 1 : 0;
+      kept += __popc(__ballot_sync(0xffffffffu, keep));
+      if (v > best) {  // lane-local first maximum
+        best = v;
+        best_j = J;
+      }
+    }
+    if (kept == 0) {
+      // the row's largest share, lowest J on ties
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, best_j, o);
+        if (ob > best || (ob == best && oj < best_j)) {
+          best = ob;
+          best_j = oj;
+        }
+      }
+      if (lane == 0) brow[best_j] = 1;
+      kept = 1;
     }
     if (lane == 0) counts[row] = kept;
   }
@@ -183,6 +245,27 @@ inline unsigned grid_for(int64_t work, int per_block, int num_sms, int max_per_s
 
 }  // namespace
 
+namespace {
+
+// row_ptr / col_idx (and the transposed CSR when requested) from the bitmap and counts
+cudaError_t csr_from_bitmap(const uint8_t* bitmap, int32_t* counts, int BH, int nb,
+                            int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                            int32_t* counts_t, int32_t* col_ptr_t, int32_t* row_idx_t,
+                            int num_sms, cudaStream_t stream) {
+  const int rows = BH * nb;
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr, nnz_out);
+  fill_kernel<<<grid_for(rows, 8, num_sms, 16), 256, 0, stream>>>(bitmap, row_ptr, rows, nb, col_idx);
+  if (col_ptr_t != nullptr && row_idx_t != nullptr) {
+    tcount_kernel<<<grid_for(rows, 256, num_sms, 8), 256, 0, stream>>>(bitmap, BH, nb, counts_t);
+    scan_kernel<<<1, 1024, 0, stream>>>(counts_t, rows, col_ptr_t, nullptr);
+    tfill_kernel<<<grid_for(rows, 256, num_sms, 8), 256, 0, stream>>>(bitmap, col_ptr_t, BH, nb,
+                                                                     row_idx_t);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uint8_t* bitmap,
                               int32_t* counts, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
                               int32_t* counts_t, int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,
@@ -195,15 +278,22 @@ cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uin
       p_imp, rows, nb, tau, bitmap, counts);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr, nnz_out);
-  fill_kernel<<<grid_for(rows, 8, num_sms, 16), 256, 0, stream>>>(bitmap, row_ptr, rows, nb, col_idx);
-  if (col_ptr_t != nullptr && row_idx_t != nullptr) {
-    tcount_kernel<<<grid_for(rows, 256, num_sms, 8), 256, 0, stream>>>(bitmap, BH, nb, counts_t);
-    scan_kernel<<<1, 1024, 0, stream>>>(counts_t, rows, col_ptr_t, nullptr);
-    tfill_kernel<<<grid_for(rows, 256, num_sms, 8), 256, 0, stream>>>(bitmap, col_ptr_t, BH, nb,
-                                                                     row_idx_t);
-  }
-  return cudaGetLastError();
+  return csr_from_bitmap(bitmap, counts, BH, nb, row_ptr, col_idx, nnz_out, counts_t, col_ptr_t,
+                         row_idx_t, num_sms, stream);
+}
+
+cudaError_t launch_build_mask_stat(const float* p_imp, int BH, int nb, double z, bool keep_all,
+                                   uint8_t* bitmap, int32_t* counts, int32_t* row_ptr,
+                                   int32_t* col_idx, int32_t* nnz_out, int32_t* counts_t,
+                                   int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,
+                                   cudaStream_t stream) {
+  const int rows = BH * nb;
+  stat_rows_kernel<<<grid_for(rows, kMaskWarps, num_sms, 16), kMaskWarps * 32, 0, stream>>>(
+      p_imp, rows, nb, z, keep_all ? 1 : 0, bitmap, counts);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return csr_from_bitmap(bitmap, counts, BH, nb, row_ptr, col_idx, nnz_out, counts_t, col_ptr_t,
+                         row_idx_t, num_sms, stream);
 }
 
 }  // namespace asa
