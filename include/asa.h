@@ -205,8 +205,8 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
 size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window);
 
 /*
- * Backward of ASA under the fixed mask (Video-BLADE, "Step 2.1": the mask restricts
- * attention "during both training and inference"; it is not differentiated):
+ * Backward of ASA under the fixed mask (Video-BLADE, "Step 2.1": the same block mask
+ * applies in training as at inference; it is not differentiated):
  *   P = exp(S - LSE), dP = dO V^T, D = rowsum(P * dP), dS = P * (dP - D),
  *   dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), dV = P^T dO, all over kept tiles only.
  * global_window = n > 0: the backward of ASA_G ("Step 2.2", variant 2, the forward

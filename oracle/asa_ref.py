@@ -7,8 +7,8 @@ Video Generation" (arXiv 2508.10774), section "Adaptive Block-Sparse Attention":
   * "Step 2.1: Sparse mask construction"            -> build_mask
   * "Step 2.2: Computation", variant 1 (standard ASA) and variant 2 (ASA_G, global
     tokens with the fixed additive ln(n) mask)      -> asa_forward
-  * the mask also restricts attention "during both training and inference" (end
-    of Step 2.1)                                    -> asa_backward (fixed mask; ASA
+  * the block mask applies in training as well as at inference (end of
+    Step 2.1)                                    -> asa_backward (fixed mask; ASA
     and ASA_G)
   * "Implementation details": b = 128, k = 16.
 
