@@ -32,6 +32,15 @@ Parity status per function (how each is pinned is in tests/test_oracle_*.py):
   build_mask_stat    pinned: k = n/2 keeps exactly the shares >= 1/n (U(1/2) = 0);
                      normal-distributed shares keep about k of n blocks (a flipped
                      quantile keeps n - k); the all-below fallback; k >= n keeps all.
+  prune_queries      pinned (BSA query pruning): a hand-computed block with known
+                     angles; the printed count of the BSA page's worked example
+                     (23,296 queries, r = 0.5 -> 11,648); cosine vs torch's
+                     cosine_similarity; brute-force maximal dissimilarity sum on tiny
+                     blocks; r = 1 and w = 1 keep all; parallel queries keep the
+                     centres and the lowest positions.
+  asa_forward_pruned pinned: torch SDPA fp64 with the token mask, rows gathered by src.
+  asa_backward_pruned pinned: torch.autograd of (masked SDPA, then the row gather by
+                     src), ASA and ASA_G.
 """
 from .gilbert import gilbert_order  # noqa: F401
 from .asa_ref import (  # noqa: F401
@@ -52,4 +61,15 @@ from .asa_ref import (  # noqa: F401
     asa_forward,
     asa_backward,
     attention_flops,
+)
+from .query_prune import (  # noqa: F401
+    window_centres,
+    kept_count,
+    cosine,
+    prune_block,
+    prune_queries,
+    marginal_tokens,
+    asa_forward_pruned,
+    filled_dout,
+    asa_backward_pruned,
 )
