@@ -74,6 +74,21 @@ def _kept_tile_flops(row_ptr, col_idx, B, H, N, d):
     return int(4 * d * (L[rows_I] * per_row).sum()), int(rp[-1]), B * H * nb * nb
 
 
+def _pruned_flops(row_ptr, col_idx, src_pos, B, H, N, d):
+    """Effective forward FLOPs with query pruning: 4 d sum over kept (I, J) of K_I L_J,
+    K_I the kept queries of block I."""
+    nb = -(-N // 128)
+    L = np.array([min(128, N - 128 * i) for i in range(nb)], dtype=np.int64)
+    kept = (src_pos.reshape(B * H, N) == np.arange(N)[None]).astype(np.int64)
+    K = np.add.reduceat(kept, np.arange(0, N, 128), axis=1).reshape(-1)      # [B*H*nb]
+    rp = row_ptr.astype(np.int64)
+    counts = np.diff(rp)
+    LJ = L[col_idx[:rp[-1]].astype(np.int64)]
+    per_row = np.add.reduceat(LJ, rp[:-1]) if rp[-1] > 0 else np.zeros(len(counts), np.int64)
+    per_row = np.where(counts > 0, per_row, 0)
+    return int(4 * d * (K * per_row).sum()), int(kept.sum())
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the GPU is busy."""
 
@@ -627,7 +642,30 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
     bwd_g_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, og, dout, lg, tmask,
                                                       global_window=64), reps=5)
     G = -(-N // 64)
+    # query pruning with token filling (r = 0.5, windows of 8) on the same mask
+    pr = asa.asa_prune_queries(qp, 0.5, 8)
+    pmws = asa._workspace(asa.lib().asa_prune_mask_workspace_size(B, H, N, pr.pack), dev)
+    ptm = asa.asa_prune_mask(tmask, pr.pack, workspace=pmws)
+    pws = asa.fwd_pruned_workspace(B, H, N, d, pr.pack, 0, dev)
+    po, plse = torch.empty_like(qp), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    prune_ms = timeit(lambda: asa.asa_prune_queries(qp, 0.5, 8, out=pr))
+    pmask_ms = timeit(lambda: asa.asa_prune_mask(tmask, pr.pack, workspace=pmws, out=ptm))
+    pfwd_ms = timeit(lambda: asa.asa_sparse_attn_fwd_pruned(pr, kp, vp, ptm, workspace=pws,
+                                                             out=po, lse=plse))
+    fwd_ms = timeit(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, tmask))
+    pflops, nkept = _pruned_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
+                                  pr.src_pos.cpu().numpy(), B, H, N, d)
+    union = int(ptm.nnz.item())
+    asa.asa_check_device_status()
     return {
+        "pruned_r0.5_w8": {
+            "pack": pr.pack, "kept_queries": nkept, "of": B * H * N,
+            "tile_entries": union, "block_entries": int(tmask.nnz.item()),
+            "prune_ms": prune_ms, "prune_mask_ms": pmask_ms, "fwd_ms": pfwd_ms,
+            "fwd_effective_tflops": pflops / pfwd_ms / 1e9,
+            "unpruned_fwd_ms": fwd_ms,
+            "speedup_total": fwd_ms / (prune_ms + pmask_ms + pfwd_ms),
+        },
         "dense_ours_fwd_ms": ours_dense, "dense_ours_tflops": dense_flops / ours_dense / 1e9,
         "dense_torch_sdpa_ms": sdpa, "dense_torch_sdpa_tflops": dense_flops / sdpa / 1e9,
         "asa_g_fwd_ms_n64": g_ms,

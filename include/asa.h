@@ -232,6 +232,104 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
                         int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
                         void* dv, void* stream);
 
+/* ------------------------------------------------------------------------------
+ * Query pruning with token filling ("Bidirectional Sparse Attention for Faster
+ * Video Diffusion Training", section "Key designs", item 1), layered on ASA's
+ * blocks of 128 permuted tokens.
+ *
+ * A block of L tokens is cut into windows of `window` consecutive permuted tokens
+ * from the block start (the last one ragged); the centre of a window of length l
+ * starting at s is token s + l/2.  The block keeps K = max(ceil(r L), windows)
+ * queries: every centre, then the other tokens with the largest 1 - cos(q_centre,
+ * q_i) to their own window's centre (ties to the lower position; a norm below 1e-8
+ * counts as 1e-8; ceil(r L) is taken in double on the float r).  Attention is
+ * computed for kept queries only; a pruned token takes its centre's output row and
+ * LSE.  In the backward a pruned token's output gradient is added to its centre's
+ * and it gets no gradient of its own.
+ *
+ * Kept queries live in a compact buffer q_s [B, H, Ns, d] of 128-row tiles: tile t
+ * holds blocks t*pack .. t*pack+pack-1, block I in rows (I % pack) * 128/pack + j of
+ * its tile (its j-th kept query in position order; unused rows zero).  One tile runs
+ * over the union of its blocks' kept key blocks (asa_prune_mask); a union entry is
+ * seen only by the 32-row lane quarters of the blocks that keep it.
+ * ---------------------------------------------------------------------------- */
+
+/* Largest pack in {1, 2, 4} whose slots (128/pack rows) hold every block's kept
+ * queries for this r and window; ASA_ERR_INVALID_ARG for r outside [0, 1] or window
+ * outside [1, 128]. */
+int asa_prune_pack(float r, int window);
+
+/* Ns = ceil(ceil(N/128) / pack) * 128 (rows per head of q_s), or a negative code. */
+int asa_prune_rows(int N, int pack);
+
+/*
+ * Selects the kept queries and packs them.  qp: device bf16 [B, H, N, d] (permuted
+ * layout); q_s: device bf16 [B, H, Ns, d], fully written (zeros in unused rows);
+ * src_pos: device int32 [B, H, N], the permuted position whose output token i
+ * takes (i if kept, else its window centre); src_row: device int32 [B, H, N], the
+ * row of q_s (and of the pruned forward's compact output) holding it.  pack must be
+ * in {1, 2, 4} and at most asa_prune_pack(r, window).
+ */
+int asa_prune_queries(const void* qp, int B, int H, int N, int d, int block, float r, int window,
+                      int pack, void* q_s, int32_t* src_pos, int32_t* src_row, void* stream);
+
+/* Workspace bytes of asa_prune_mask (a count per tile), 0 for invalid sizes. */
+size_t asa_prune_mask_workspace_size(int B, int H, int N, int pack);
+
+/*
+ * Tile CSR of the packed queries from a block mask (row_ptr/col_idx of
+ * asa_build_mask or asa_build_mask_stat): tile_ptr [B*H*ntile + 1] (ntile =
+ * ceil(ceil(N/128)/pack)), tile_col [capacity nnz of the input] ascending key
+ * blocks of the union, tile_quarters [same] with bit q set when lane quarter q
+ * (rows 32q .. 32q+31 of the tile) belongs to a block that keeps that key block;
+ * nnz_out: device int32, the union's entry count.  An input column outside
+ * [0, ceil(N/128)) is skipped and reported by asa_check_device_status as
+ * ASA_ERR_INVALID_ARG.
+ */
+int asa_prune_mask(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N, int pack,
+                   void* workspace, size_t ws_bytes, int32_t* tile_ptr, int32_t* tile_col,
+                   uint8_t* tile_quarters, int32_t* nnz_out, void* stream);
+
+/* Workspace bytes of asa_sparse_attn_fwd_pruned: the tile launch order, the compact
+ * output (bf16 [B, H, Ns, d]) and LSE (fp32 [B, H, Ns]), the ASA_G global tokens. */
+size_t asa_fwd_pruned_workspace_size(int B, int H, int N, int d, int pack, int global_window);
+
+/*
+ * Step 2.2 (ASA, or ASA_G with global_window = n > 0) for the kept queries only,
+ * then token filling: o [B, H, N, d] bf16 and lse [B, H, N] fp32 take, for every
+ * token i, the compact row src_row[i].  q_s, src_row: from asa_prune_queries; kp,
+ * vp: the full permuted keys and values; tile_*: from asa_prune_mask.  A src_row
+ * outside [0, Ns) writes a zero row, lse -inf, and is reported as
+ * ASA_ERR_INVALID_ARG by asa_check_device_status.
+ */
+int asa_sparse_attn_fwd_pruned(const void* q_s, const void* kp, const void* vp,
+                               const int32_t* tile_ptr, const int32_t* tile_col,
+                               const uint8_t* tile_quarters, const int32_t* src_row, int B, int H,
+                               int N, int d, int block, int pack, int global_window,
+                               void* workspace, size_t ws_bytes, void* o, float* lse,
+                               void* stream);
+
+/* Workspace bytes of asa_sparse_attn_bwd_pruned: asa_bwd_workspace_size plus the
+ * gathered output gradient (bf16 [B, H, N, d]) and the row LSEs (fp32 [B, H, N]). */
+size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int global_window);
+
+/*
+ * Backward with query pruning under the fixed mask: with dO'[c] = the sum of dO[i]
+ * over the tokens i with src_pos[i] = c (stored in bf16; zero on pruned rows) it
+ * computes asa_sparse_attn_bwd's gradients for the kept rows, and pruned rows get
+ * dQ = 0 (their LSE is taken as +inf, so their probabilities vanish).  Inputs as in
+ * asa_sparse_attn_bwd, with lse the pruned forward's and src_pos from
+ * asa_prune_queries (each token must map to a token of its own block that maps to
+ * itself; other rows are zeroed and reported as ASA_ERR_INVALID_ARG).  The kept
+ * rows run in the full layout: the backward does the unpruned amount of work.
+ */
+int asa_sparse_attn_bwd_pruned(const void* qp, const void* kp, const void* vp, const void* dout,
+                               const float* lse, const int32_t* src_pos, const int32_t* row_ptr,
+                               const int32_t* col_idx, const int32_t* col_ptr_t,
+                               const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                               int global_window, void* workspace, size_t ws_bytes, void* dq,
+                               void* dk, void* dv, void* stream);
+
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of
  * the current device.  Returns ASA_OK, ASA_ERR_TIMEOUT if a kernel gave up a

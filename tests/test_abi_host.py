@@ -158,3 +158,64 @@ def test_workspace_sizes(L):
     assert extra >= 12 * G * 128 * (3 * 2 + 2 * 4)
     assert L.asa_bwd_workspace_size(1, 12, 32760, 128, -1) == 0
     assert L.asa_estimate_mask_workspace_size(0, 12, 32760) == 0
+
+
+def test_prune_host_rules(L):
+    # pack: 4 while a block keeps at most 32 queries, 2 up to 64, else 1
+    assert L.asa_prune_pack(0.5, 8) == 2
+    assert L.asa_prune_pack(0.25, 8) == 4
+    assert L.asa_prune_pack(0.25, 2) == 2        # 64 centres per block
+    assert L.asa_prune_pack(0.51, 8) == 1
+    assert L.asa_prune_pack(0.0, 128) == 4
+    assert L.asa_prune_pack(1.5, 8) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_prune_pack(float("nan"), 8) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_prune_pack(0.5, 0) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_prune_pack(0.5, 129) == asa.ASA_ERR_INVALID_ARG
+    # compact rows: whole tiles of `pack` blocks
+    assert L.asa_prune_rows(32760, 2) == 128 * 128
+    assert L.asa_prune_rows(300, 4) == 128
+    assert L.asa_prune_rows(300, 1) == 3 * 128
+    assert L.asa_prune_rows(300, 3) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_prune_rows(0, 1) == asa.ASA_ERR_INVALID_ARG
+
+
+def test_prune_rejects(L):
+    q = lambda pack=2, r=0.5, w=8, qp=FAKE, d=64: L.asa_prune_queries(
+        qp, 1, 2, 1024, d, 128, r, w, pack, FAKE, FAKE, FAKE, None)
+    assert q(pack=4) == asa.ASA_ERR_INVALID_ARG     # 64 kept rows do not fit 32-row slots
+    assert q(pack=3) == asa.ASA_ERR_INVALID_ARG
+    assert q(r=-0.1) == asa.ASA_ERR_INVALID_ARG
+    assert q(w=0) == asa.ASA_ERR_INVALID_ARG
+    assert q(qp=MIS) == asa.ASA_ERR_INVALID_ARG
+    assert q(d=96) == asa.ASA_ERR_UNSUPPORTED
+    assert b"pack" in (q(pack=4) and L.asa_last_error_string())
+    # the tile CSR needs its counts workspace
+    assert L.asa_prune_mask(FAKE, FAKE, 1, 2, 1024, 2, None, 0, FAKE, FAKE, FAKE, FAKE,
+                            None) == asa.ASA_ERR_WORKSPACE
+    assert L.asa_prune_mask(FAKE, FAKE, 1, 2, 1024, 2, None, 0, FAKE, FAKE, None, FAKE,
+                            None) == asa.ASA_ERR_INVALID_ARG
+    fwd = [FAKE] * 7 + [1, 2, 1024, 64, 128, 2, 0, None, 0, FAKE, FAKE, None]
+    assert L.asa_sparse_attn_fwd_pruned(*fwd) == asa.ASA_ERR_WORKSPACE
+    fwd[12] = 3      # pack
+    assert L.asa_sparse_attn_fwd_pruned(*fwd) == asa.ASA_ERR_INVALID_ARG
+    fwd[12] = 2
+    fwd[13] = -1     # global_window
+    assert L.asa_sparse_attn_fwd_pruned(*fwd) == asa.ASA_ERR_INVALID_ARG
+    bwd = [FAKE] * 10 + [1, 2, 1024, 64, 128, 0, None, 0] + [FAKE] * 3 + [None]
+    assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_WORKSPACE
+    bwd[5] = None    # src_pos
+    assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_INVALID_ARG
+
+
+def test_prune_workspace_sizes(L):
+    BH, N, d = 12, 32760, 128
+    tiles = BH * 128                     # 256 blocks, 2 per tile
+    assert L.asa_prune_mask_workspace_size(1, 12, N, 2) >= tiles * 4
+    assert L.asa_prune_mask_workspace_size(1, 12, N, 3) == 0
+    fw = L.asa_fwd_pruned_workspace_size(1, 12, N, d, 2, 0)
+    assert fw >= tiles * 4 + tiles * 128 * (d * 2 + 4)      # order, compact O and LSE
+    G = -(-N // 64)
+    assert L.asa_fwd_pruned_workspace_size(1, 12, N, d, 2, 64) - fw >= 2 * BH * G * d * 2
+    bw = L.asa_bwd_pruned_workspace_size(1, 12, N, d, 0)
+    assert bw >= L.asa_bwd_workspace_size(1, 12, N, d, 0) + BH * N * (d * 2 + 4)
+    assert L.asa_bwd_pruned_workspace_size(1, 12, N, 96, 0) == 0

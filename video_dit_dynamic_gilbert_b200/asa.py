@@ -44,6 +44,15 @@ _SIGNATURES = {
     "asa_bwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_build_mask_stat": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size] + [_vp] * 6, _c_int),
+    "asa_prune_pack": ([_c_float, _c_int], _c_int),
+    "asa_prune_rows": ([_c_int, _c_int], _c_int),
+    "asa_prune_queries": ([_vp] + [_c_int] * 5 + [_c_float, _c_int, _c_int] + [_vp] * 4, _c_int),
+    "asa_prune_mask_workspace_size": ([_c_int] * 4, _c_size),
+    "asa_prune_mask": ([_vp, _vp] + [_c_int] * 4 + [_vp, _c_size] + [_vp] * 5, _c_int),
+    "asa_fwd_pruned_workspace_size": ([_c_int] * 6, _c_size),
+    "asa_sparse_attn_fwd_pruned": ([_vp] * 7 + [_c_int] * 7 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
+    "asa_bwd_pruned_workspace_size": ([_c_int] * 5, _c_size),
+    "asa_sparse_attn_bwd_pruned": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),
@@ -317,6 +326,140 @@ def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, global_window
     return outs
 
 
+# ----------------------------------------------------------------------- query pruning (BSA)
+
+@dataclass
+class QueryPrune:
+    """Kept queries packed into 128-row tiles (q_s [B, H, Ns, d]) and, per token, the
+    permuted position (src_pos) and compact row (src_row) whose output it takes."""
+    q_s: torch.Tensor
+    src_pos: torch.Tensor
+    src_row: torch.Tensor
+    pack: int
+    r: float
+    window: int
+    N: int
+
+    @property
+    def Ns(self) -> int:
+        return self.q_s.shape[2]
+
+
+@dataclass
+class TileMask:
+    """CSR over the packed query tiles: the union of the tile's blocks' kept key blocks,
+    with the 32-row lane quarters that see each entry."""
+    tile_ptr: torch.Tensor
+    tile_col: torch.Tensor
+    tile_quarters: torch.Tensor
+    nnz: torch.Tensor
+    pack: int
+
+
+def asa_prune_pack(r: float, window: int) -> int:
+    """Largest tile packing (1, 2 or 4 blocks per 128-row tile) this r and window allow."""
+    rc = lib().asa_prune_pack(float(r), int(window))
+    _check(min(rc, 0))
+    return rc
+
+
+def asa_prune_rows(N: int, pack: int) -> int:
+    rc = lib().asa_prune_rows(int(N), int(pack))
+    _check(min(rc, 0))
+    return rc
+
+
+def asa_prune_queries(qp: torch.Tensor, r: float, window: int = 8, pack: int = 0,
+                      out: QueryPrune | None = None, stream=None) -> QueryPrune:
+    """Query pruning (BSA): keep every window centre and the queries least similar to
+    their centre, K = max(ceil(r L), windows) per block; pack = 0 takes the largest
+    packing allowed."""
+    _bf16_cuda("qp", qp)
+    B, H, N, d = qp.shape
+    if pack == 0:
+        pack = asa_prune_pack(r, window)
+    Ns = asa_prune_rows(N, pack)
+    if out is None:
+        z = dict(dtype=torch.int32, device=qp.device)
+        out = QueryPrune(torch.empty((B, H, Ns, d), dtype=qp.dtype, device=qp.device),
+                         torch.empty((B, H, N), **z), torch.empty((B, H, N), **z), pack,
+                         float(r), int(window), N)
+    _check(lib().asa_prune_queries(_ptr(qp), B, H, N, d, BLOCK, float(r), int(window), pack,
+                                   _ptr(out.q_s), _ptr(out.src_pos), _ptr(out.src_row),
+                                   _stream(stream)))
+    return out
+
+
+def asa_prune_mask(mask: BlockMask, pack: int, workspace=None, out: TileMask | None = None,
+                   stream=None) -> TileMask:
+    """Tile CSR of the packed queries from a block mask."""
+    B, H, N = mask.B, mask.H, mask.N
+    dev = mask.row_ptr.device
+    if workspace is None:
+        workspace = _workspace(lib().asa_prune_mask_workspace_size(B, H, N, pack), dev)
+    if out is None:
+        tiles = B * H * -(-nblocks(N) // pack)
+        cap = mask.col_idx.numel()
+        z = dict(dtype=torch.int32, device=dev)
+        out = TileMask(torch.empty(tiles + 1, **z), torch.empty(cap, **z),
+                       torch.empty(cap, dtype=torch.uint8, device=dev), torch.empty(1, **z), pack)
+    _check(lib().asa_prune_mask(_ptr(mask.row_ptr), _ptr(mask.col_idx), B, H, N, pack,
+                                _ptr(workspace), _ws_bytes(workspace), _ptr(out.tile_ptr),
+                                _ptr(out.tile_col), _ptr(out.tile_quarters), _ptr(out.nnz),
+                                _stream(stream)))
+    return out
+
+
+def fwd_pruned_workspace(B, H, N, d, pack, global_window, device):
+    return _workspace(lib().asa_fwd_pruned_workspace_size(B, H, N, d, pack, global_window), device)
+
+
+def asa_sparse_attn_fwd_pruned(prune: QueryPrune, kp, vp, tmask: TileMask, global_window: int = 0,
+                               workspace=None, out=None, lse=None, stream=None):
+    """Forward for the kept queries only, then token filling: O [B, H, N, d] bf16 and
+    LSE [B, H, N] fp32 (a pruned token takes its centre's row)."""
+    for n_, t in (("kp", kp), ("vp", vp)):
+        _bf16_cuda(n_, t)
+    B, H, N, d = kp.shape
+    if workspace is None:
+        workspace = fwd_pruned_workspace(B, H, N, d, prune.pack, global_window, kp.device)
+    if out is None:
+        out = torch.empty_like(kp)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=kp.device)
+    _check(lib().asa_sparse_attn_fwd_pruned(
+        _ptr(prune.q_s), _ptr(kp), _ptr(vp), _ptr(tmask.tile_ptr), _ptr(tmask.tile_col),
+        _ptr(tmask.tile_quarters), _ptr(prune.src_row), B, H, N, d, BLOCK, prune.pack,
+        global_window, _ptr(workspace), _ws_bytes(workspace), _ptr(out), _ptr(lse),
+        _stream(stream)))
+    return out, lse
+
+
+def bwd_pruned_workspace(B, H, N, d, device, global_window: int = 0):
+    return _workspace(lib().asa_bwd_pruned_workspace_size(B, H, N, d, global_window), device)
+
+
+def asa_sparse_attn_bwd_pruned(qp, kp, vp, dout, lse, mask: BlockMask, prune: QueryPrune,
+                               global_window: int = 0, workspace=None, outs=None, stream=None):
+    """dQ, dK, dV [B, H, N, d] bf16 with query pruning under the fixed mask: pruned
+    tokens' output gradients go to their centres; pruned rows get dQ = 0."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp), ("dout", dout)):
+        _bf16_cuda(n_, t)
+    if mask.col_ptr_t is None:
+        raise ValueError("the backward needs the transposed CSR (transposed=True)")
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = bwd_pruned_workspace(B, H, N, d, qp.device, global_window)
+    if outs is None:
+        outs = tuple(torch.empty_like(qp) for _ in range(3))
+    _check(lib().asa_sparse_attn_bwd_pruned(
+        _ptr(qp), _ptr(kp), _ptr(vp), _ptr(dout), _ptr(lse), _ptr(prune.src_pos),
+        _ptr(mask.row_ptr), _ptr(mask.col_idx), _ptr(mask.col_ptr_t), _ptr(mask.row_idx_t),
+        B, H, N, d, BLOCK, global_window, _ptr(workspace), _ws_bytes(workspace),
+        *(_ptr(t) for t in outs), _stream(stream)))
+    return outs
+
+
 def asa_check_device_status(stream=None) -> None:
     _check(lib().asa_check_device_status(_stream(stream)))
 
@@ -333,12 +476,20 @@ def asa_shutdown() -> None:
 # ----------------------------------------------------------------------- one attention call
 
 def asa_attention(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
-                  stream=None):
+                  query_keep: float | None = None, query_window: int = 8, stream=None):
     """One ASA self-attention call on raster-layout q, k, v [B, N, H, d]: Gilbert permute,
-    estimate + mask, block-sparse forward, unpermute.  Returns (O raster, LSE, mask)."""
+    estimate + mask, block-sparse forward, unpermute.  Returns (O raster, LSE, mask).
+    query_keep = r adds BSA's query pruning with token filling (windows of
+    query_window permuted tokens)."""
     qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W, stream=stream)
     mask = asa_estimate_mask(qp, kp, tau, transposed=False, stream=stream)
-    op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window, stream=stream)
+    if query_keep is None:
+        op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window, stream=stream)
+    else:
+        prune = asa_prune_queries(qp, query_keep, query_window, stream=stream)
+        tmask = asa_prune_mask(mask, prune.pack, stream=stream)
+        op, lse = asa_sparse_attn_fwd_pruned(prune, kp, vp, tmask, global_window=global_window,
+                                             stream=stream)
     return asa_unpermute(op, T, Hg, W, stream=stream), lse, mask
 
 
@@ -349,13 +500,20 @@ class ASAAttention(torch.autograd.Function):
     asa_sparse_attn_bwd under that mask, its gradients unpermuted to raster layout."""
 
     @staticmethod
-    def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0):
+    def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
+                query_keep: float | None = None, query_window: int = 8):
         q, k, v = (t.contiguous() for t in (q, k, v))
         qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W)
         mask = asa_estimate_mask(qp, kp, tau, transposed=True)
-        op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window)
+        prune = None
+        if query_keep is None:
+            op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window)
+        else:
+            prune = asa_prune_queries(qp, query_keep, query_window)
+            tmask = asa_prune_mask(mask, prune.pack)
+            op, lse = asa_sparse_attn_fwd_pruned(prune, kp, vp, tmask, global_window=global_window)
         ctx.save_for_backward(qp, kp, vp, op, lse)
-        ctx.mask, ctx.grid, ctx.global_window = mask, (T, Hg, W), global_window
+        ctx.mask, ctx.grid, ctx.global_window, ctx.prune = mask, (T, Hg, W), global_window, prune
         return asa_unpermute(op, T, Hg, W)
 
     @staticmethod
@@ -363,15 +521,21 @@ class ASAAttention(torch.autograd.Function):
         qp, kp, vp, op, lse = ctx.saved_tensors
         T, Hg, W = ctx.grid
         dop = asa_gilbert_permute(dout.to(torch.bfloat16).contiguous(), T, Hg, W)
-        grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
-                                    global_window=ctx.global_window)
+        if ctx.prune is None:
+            grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
+                                        global_window=ctx.global_window)
+        else:
+            grads = asa_sparse_attn_bwd_pruned(qp, kp, vp, dop, lse, ctx.mask, ctx.prune,
+                                               global_window=ctx.global_window)
         dq, dk, dv = (asa_unpermute(g, T, Hg, W) for g in grads)
-        return dq, dk, dv, None, None, None, None, None
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
 def asa_attention_trainable(q, k, v, T: int, Hg: int, W: int, tau: float,
-                            global_window: int = 0):
+                            global_window: int = 0, query_keep: float | None = None,
+                            query_window: int = 8):
     """Differentiable asa_attention: returns O [B, N, H, d] (raster); gradients flow to
-    q, k and v through the kernels' backward under the forward's mask."""
-    return ASAAttention.apply(q, k, v, T, Hg, W, tau, global_window)
+    q, k and v through the kernels' backward under the forward's mask (and, with
+    query_keep, the forward's query pruning)."""
+    return ASAAttention.apply(q, k, v, T, Hg, W, tau, global_window, query_keep, query_window)
 

@@ -4,6 +4,7 @@
 // anything, carves the caller's workspace, and launches the kernels of its step on
 // the caller's stream.  The only memory the library owns is the per-shape Gilbert
 // permutation table (built on the host once per (device, T, Hg, W) and uploaded).
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -463,6 +464,212 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
   return ASA_OK;
 }
 
+// ---------------------------------------------------------------- query pruning (BSA)
+
+namespace {
+
+int prune_kept_max(float r, int window) {
+  return std::max(static_cast<int>(std::ceil(static_cast<double>(r) * ASA_BLOCK)),
+                  (ASA_BLOCK + window - 1) / window);
+}
+
+int check_prune(float r, int window) {
+  if (!(r >= 0.f && r <= 1.f)) return fail(ASA_ERR_INVALID_ARG, "keep ratio r=%g not in [0, 1]", r);
+  if (window < 1 || window > ASA_BLOCK)
+    return fail(ASA_ERR_INVALID_ARG, "window=%d not in [1, %d]", window, ASA_BLOCK);
+  return ASA_OK;
+}
+
+int check_pack(int pack) {
+  if (pack != 1 && pack != 2 && pack != 4)
+    return fail(ASA_ERR_INVALID_ARG, "pack=%d not in {1, 2, 4}", pack);
+  return ASA_OK;
+}
+
+size_t prune_tiles(int B, int H, int N, int pack) {
+  const size_t nb = (static_cast<size_t>(N) + ASA_BLOCK - 1) / ASA_BLOCK;
+  return static_cast<size_t>(B) * H * ((nb + pack - 1) / pack);
+}
+
+}  // namespace
+
+int asa_prune_pack(float r, int window) {
+  ASA_TRY(check_prune(r, window));
+  const int k = prune_kept_max(r, window);
+  return k <= ASA_BLOCK / 4 ? 4 : (k <= ASA_BLOCK / 2 ? 2 : 1);
+}
+
+int asa_prune_rows(int N, int pack) {
+  if (N < 1 || N > ASA_MAX_TOKENS) return fail(ASA_ERR_INVALID_ARG, "N=%d not in [1, %d]", N, ASA_MAX_TOKENS);
+  ASA_TRY(check_pack(pack));
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  return (nb + pack - 1) / pack * ASA_BLOCK;
+}
+
+int asa_prune_queries(const void* qp, int B, int H, int N, int d, int block, float r, int window,
+                      int pack, void* q_s, int32_t* src_pos, int32_t* src_row, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  ASA_TRY(check_prune(r, window));
+  ASA_TRY(check_pack(pack));
+  if (pack > asa_prune_pack(r, window))
+    return fail(ASA_ERR_INVALID_ARG, "pack=%d: a block keeps up to %d queries, more than 128/%d",
+                pack, prune_kept_max(r, window), pack);
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(q_s, "q_s"));
+  ASA_TRY(check_ptr(src_pos, "src_pos", false));
+  ASA_TRY(check_ptr(src_row, "src_row", false));
+  const int Ns = asa_prune_rows(N, pack);
+  cudaError_t e = asa::launch_prune(qp, B * H, N, d, r, window, pack, q_s, Ns, src_pos, src_row,
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prune launch");
+  return ASA_OK;
+}
+
+size_t asa_prune_mask_workspace_size(int B, int H, int N, int pack) {
+  if (B < 1 || H < 1 || N < 1 || N > ASA_MAX_TOKENS || (pack != 1 && pack != 2 && pack != 4))
+    return 0;
+  return align256(prune_tiles(B, H, N, pack) * sizeof(int32_t));
+}
+
+int asa_prune_mask(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N, int pack,
+                   void* workspace, size_t ws_bytes, int32_t* tile_ptr, int32_t* tile_col,
+                   uint8_t* tile_quarters, int32_t* nnz_out, void* stream) {
+  ASA_TRY(check_common(B, H, N, 64));
+  ASA_TRY(check_pack(pack));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(tile_ptr, "tile_ptr", false));
+  ASA_TRY(check_ptr(tile_col, "tile_col", false));
+  if (tile_quarters == nullptr) return fail(ASA_ERR_INVALID_ARG, "tile_quarters is NULL");
+  ASA_TRY(check_ptr(nnz_out, "nnz_out", false));
+  ASA_TRY(check_ws(workspace, ws_bytes, asa_prune_mask_workspace_size(B, H, N, pack)));
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  const int nb = (N + ASA_BLOCK - 1) / ASA_BLOCK;
+  e = asa::launch_prune_mask(row_ptr, col_idx, B * H, nb, pack, static_cast<int32_t*>(workspace),
+                             tile_ptr, tile_col, tile_quarters, nnz_out, err_word,
+                             num_sms_current(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prune mask launch");
+  return ASA_OK;
+}
+
+size_t asa_fwd_pruned_workspace_size(int B, int H, int N, int d, int pack, int global_window) {
+  if (B < 1 || H < 1 || N < 1 || N > ASA_MAX_TOKENS || (d != 64 && d != 128) ||
+      (pack != 1 && pack != 2 && pack != 4) || global_window < 0)
+    return 0;
+  const size_t tiles = prune_tiles(B, H, N, pack);
+  const size_t rows = tiles * ASA_BLOCK;  // B*H*Ns
+  size_t bytes = align256(tiles * sizeof(int32_t)) + align256(rows * d * 2) +
+                 align256(rows * sizeof(float));
+  if (global_window > 0) {
+    const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    bytes += 2 * align256(static_cast<size_t>(B) * H * G * d * 2);
+  }
+  return bytes;
+}
+
+int asa_sparse_attn_fwd_pruned(const void* q_s, const void* kp, const void* vp,
+                               const int32_t* tile_ptr, const int32_t* tile_col,
+                               const uint8_t* tile_quarters, const int32_t* src_row, int B, int H,
+                               int N, int d, int block, int pack, int global_window,
+                               void* workspace, size_t ws_bytes, void* o, float* lse,
+                               void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  ASA_TRY(check_pack(pack));
+  ASA_TRY(check_ptr(q_s, "q_s"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(vp, "vp"));
+  ASA_TRY(check_ptr(tile_ptr, "tile_ptr", false));
+  ASA_TRY(check_ptr(tile_col, "tile_col", false));
+  if (tile_quarters == nullptr) return fail(ASA_ERR_INVALID_ARG, "tile_quarters is NULL");
+  ASA_TRY(check_ptr(src_row, "src_row", false));
+  ASA_TRY(check_ptr(o, "o"));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  ASA_TRY(check_ws(workspace, ws_bytes, asa_fwd_pruned_workspace_size(B, H, N, d, pack, global_window)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const int Ns = asa_prune_rows(N, pack);
+  const size_t tiles = prune_tiles(B, H, N, pack);
+  char* p = static_cast<char*>(workspace);
+  int32_t* order = reinterpret_cast<int32_t*>(p);
+  p += align256(tiles * sizeof(int32_t));
+  void* o_s = p;
+  p += align256(tiles * ASA_BLOCK * d * 2);
+  float* lse_s = reinterpret_cast<float*>(p);
+  p += align256(tiles * ASA_BLOCK * sizeof(float));
+  const void* kg = nullptr;
+  const void* vg = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (global_window > 0) {
+    const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    void* kgw = p;
+    void* vgw = p + align256(static_cast<size_t>(BH) * G * d * 2);
+    e = asa::launch_global_pool(kp, kgw, BH, N, d, global_window, num_sms_current(), s);
+    if (e == cudaSuccess) e = asa::launch_global_pool(vp, vgw, BH, N, d, global_window, num_sms_current(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    kg = kgw;
+    vg = vgw;
+  }
+  unsigned int* err_word = nullptr;
+  e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_fwd_tc_pruned(q_s, kp, vp, tile_ptr, tile_col, tile_quarters, kg, vg, order, BH,
+                                N, Ns, d, global_window, o_s, lse_s, err_word, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pruned forward launch");
+  e = asa::launch_fill_out(o_s, lse_s, src_row, BH, N, Ns, d, o, lse, err_word, num_sms_current(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "fill launch");
+  return ASA_OK;
+}
+
+size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int global_window) {
+  const size_t base = asa_bwd_workspace_size(B, H, N, d, global_window);
+  if (base == 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return align256(base) + align256(rows * d * 2) + align256(rows * sizeof(float));
+}
+
+int asa_sparse_attn_bwd_pruned(const void* qp, const void* kp, const void* vp, const void* dout,
+                               const float* lse, const int32_t* src_pos, const int32_t* row_ptr,
+                               const int32_t* col_idx, const int32_t* col_ptr_t,
+                               const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                               int global_window, void* workspace, size_t ws_bytes, void* dq,
+                               void* dk, void* dv, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  const void* bf[] = {qp, kp, vp, dout, dq, dk, dv};
+  const char* names[] = {"qp", "kp", "vp", "dout", "dq", "dk", "dv"};
+  for (int k = 0; k < 7; ++k) ASA_TRY(check_ptr(bf[k], names[k]));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  ASA_TRY(check_ptr(src_pos, "src_pos", false));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(col_ptr_t, "col_ptr_t", false));
+  ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  ASA_TRY(check_ws(workspace, ws_bytes, asa_bwd_pruned_workspace_size(B, H, N, d, global_window)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  char* p = static_cast<char*>(workspace);
+  void* bwd_ws = p;
+  p += align256(asa_bwd_workspace_size(B, H, N, d, global_window));
+  void* dout2 = p;
+  p += align256(rows * d * 2);
+  float* lse2 = reinterpret_cast<float*>(p);
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  e = asa::launch_dout_fill(dout, lse, src_pos, B * H, N, d, dout2, lse2, err_word, num_sms_current(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "gradient fill launch");
+  e = asa::launch_bwd_tc(qp, kp, vp, dout2, lse2, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
+                         d, global_window, bwd_ws, dq, dk, dv, err_word, num_sms_current(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return ASA_OK;
+}
+
 int asa_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1 || limit_cycles > (1ll << 31))
     return fail(ASA_ERR_INVALID_ARG, "limit_cycles=%lld outside [1, 2^31]", limit_cycles);
@@ -486,6 +693,10 @@ int asa_check_device_status(void* stream) {
     if (word & 8u)
       return fail(ASA_ERR_INVALID_ARG,
                   "backward: a Q or K value is out of fp16 range (|x| > 65504) (word 0x%x)", word);
+    if (word & 32u)
+      return fail(ASA_ERR_INVALID_ARG,
+                  "an index argument (CSR column, src_pos or src_row) is out of range (word 0x%x)",
+                  word);
     return fail(ASA_ERR_TIMEOUT, "a device-side bounded wait expired (word 0x%x)", word);
   }
   return ASA_OK;

@@ -86,15 +86,18 @@ __device__ __forceinline__ TileSrc tile_src(int j, int nfine, const int32_t* col
   return t;
 }
 
-template <int D, int NST>
+// kPruned: the query tiles are packed tiles of pruned queries (Nq rows per head).
+// Entry e of the tile's CSR row is seen only by the 32-row lane quarters q with bit q
+// of quarters[e] set; the other quarters' rows give that key tile probability 0.
+template <int D, int NST, bool kPruned>
 __global__ void __launch_bounds__(kFwdTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
                   const __grid_constant__ CUtensorMap tmVg, const int32_t* __restrict__ row_ptr,
-                  const int32_t* __restrict__ col_idx, const int32_t* __restrict__ order, int N,
-                  int nb, int G, float gbias2, float c2, __nv_bfloat16* __restrict__ o,
-                  float* __restrict__ lse, unsigned int* __restrict__ err_word,
-                  long long wait_limit) {
+                  const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ quarters,
+                  const int32_t* __restrict__ order, int N, int Nq, int nb, int G, float gbias2,
+                  float c2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                  unsigned int* __restrict__ err_word, long long wait_limit) {
   using L = FwdTcLayout<D, NST>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -282,6 +285,20 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       }
       tc::fence_after();
       const TileSrc t = tile_src(j, nfine, cols, N, G);
+      if constexpr (kPruned) {
+        if (!t.global && ((quarters[rbeg + j] >> quarter) & 1u) == 0u) {
+          // these rows do not keep key block cols[j]: P = 0, running max and sum unchanged
+          uint32_t z[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) z[k] = 0u;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tc::tmem_st16(tS + 16u * c, z);
+          tc::tmem_wait_st();
+          tc::fence_before();
+          tc::mbar_arrive(p_full(w));
+          continue;
+        }
+      }
       const float bias = t.global ? gbias2 : 0.f;
       uint32_t s[128];
 #pragma unroll
@@ -374,10 +391,12 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     // merge the two streams: (m, l) through shared memory, over Q's bytes (every MMA
     // that reads Q is complete once both warpgroups hold their last PV)
     float* red = reinterpret_cast<float*>(sbase + L::kQ);  // [2][2][128]: m, l per stream
+    // with pruning a stream may hold no tile these rows see (O stays 0, m = -inf)
+    const bool live = kPruned ? (have_o && m_ref != -INFINITY) : have_o;
     tc::named_bar_sync(1, 256);
-    red[(2 * w) * 128 + row] = have_o ? m_ref : -INFINITY;
-    red[(2 * w + 1) * 128 + row] = have_o ? l : 0.f;
-    red[(4 + w) * 128 + row] = have_o ? 1.f : 0.f;
+    red[(2 * w) * 128 + row] = live ? m_ref : -INFINITY;
+    red[(2 * w + 1) * 128 + row] = live ? l : 0.f;
+    red[(4 + w) * 128 + row] = live ? 1.f : 0.f;
     tc::named_bar_sync(1, 256);
     const float m_0 = red[0 * 128 + row], l_0 = red[1 * 128 + row];
     const float m_1 = red[2 * 128 + row], l_1 = red[3 * 128 + row];
@@ -389,7 +408,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
     // warpgroup w writes columns [D/2 w, D/2 w + D/2) of its rows
     const int q = q0 + row;
-    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D + (D / 2) * w;
+    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
     const bool h0 = __all_sync(0xffffffffu, has_0) != 0 || __any_sync(0xffffffffu, has_0) != 0;
     const bool h1 = __any_sync(0xffffffffu, has_1) != 0;
 #pragma unroll
@@ -409,7 +428,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         for (int k = 0; k < 32; ++k) a1[k] = 0u;
       }
       const float f0 = s_0 * inv, f1 = s_1 * inv;
-      if (q < N) {
+      if (q < Nq) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           float x[8];
@@ -428,8 +447,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         }
       }
     }
-    if (q < N && w == 0)
-      lse[static_cast<int64_t>(bh) * N + q] = l_row > 0.f ? (m + __log2f(l_row)) * kLn2 : -INFINITY;
+    if (q < Nq && w == 0)
+      lse[static_cast<int64_t>(bh) * Nq + q] = l_row > 0.f ? (m + __log2f(l_row)) * kLn2 : -INFINITY;
   }
 
   if (failed) atomicOr(err_word, 1u);
@@ -538,21 +557,23 @@ cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
 
 namespace {
 
-template <int D, int NST>
+// Nq query rows per head in nb query tiles (N, ceil(N/128) without pruning).
+template <int D, int NST, bool kPruned>
 cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int32_t* col_idx,
-                      int32_t* order, int BH, int N, int G, float gbias2, void* o, float* lse,
-                      unsigned int* err_word, cudaStream_t stream) {
+                      const uint8_t* quarters, int32_t* order, int BH, int N, int Nq, int G,
+                      float gbias2, void* o, float* lse, unsigned int* err_word,
+                      cudaStream_t stream) {
   using L = FwdTcLayout<D, NST>;
-  const int nb = (N + kBlock - 1) / kBlock;
+  const int nb = (Nq + kBlock - 1) / kBlock;
   const float c2 = kLog2e / sqrtf(static_cast<float>(D));
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST, kPruned>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   // the register split inside the kernel assumes exactly kLaunchRegs per thread at launch
   static int regs_checked = 0;
   if (regs_checked == 0) {
     cudaFuncAttributes fa{};
-    e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<D, NST>);
+    e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<D, NST, kPruned>);
     if (e != cudaSuccess) return e;
     regs_checked = fa.numRegs == kLaunchRegs ? 1 : -1;
   }
@@ -561,22 +582,22 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   const int rows = nb * BH;
   e = launch_lpt_order(row_ptr, BH, nb, order, stream);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D, NST><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, order, N, nb, G, gbias2, c2,
-      static_cast<__nv_bfloat16*>(o), lse, err_word, limit);
+  fwd_tc_kernel<D, NST, kPruned><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, quarters, order, N, Nq, nb,
+      G, gbias2, c2, static_cast<__nv_bfloat16*>(o), lse, err_word, limit);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
-                          const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
-                          int BH, int N, int d, int global_window, void* o, float* lse,
-                          unsigned int* err_word, cudaStream_t stream) {
+template <bool kPruned>
+cudaError_t launch_fwd_any(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                           const int32_t* col_idx, const uint8_t* quarters, const void* kg,
+                           const void* vg, int32_t* order, int BH, int N, int Nq, int d,
+                           int global_window, void* o, float* lse, unsigned int* err_word,
+                           cudaStream_t stream) {
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
   const float gbias2 = global_window > 0 ? log2f(static_cast<float>(global_window)) : 0.f;
   CUtensorMap maps[5];
-  if (!make_map(&maps[0], qp, BH, N, d) || !make_map(&maps[1], kp, BH, N, d) ||
+  if (!make_map(&maps[0], qp, BH, Nq, d) || !make_map(&maps[1], kp, BH, N, d) ||
       !make_map(&maps[2], vp, BH, N, d))
     return cudaErrorInvalidValue;
   if (G > 0) {
@@ -587,8 +608,30 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
     maps[4] = maps[2];
   }
   if (d == 128)
-    return launch_tc<128, 3>(maps, row_ptr, col_idx, order, BH, N, G, gbias2, o, lse, err_word, stream);
-  return launch_tc<64, 6>(maps, row_ptr, col_idx, order, BH, N, G, gbias2, o, lse, err_word, stream);
+    return launch_tc<128, 3, kPruned>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G,
+                                      gbias2, o, lse, err_word, stream);
+  return launch_tc<64, 6, kPruned>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G, gbias2,
+                                   o, lse, err_word, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                          const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
+                          int BH, int N, int d, int global_window, void* o, float* lse,
+                          unsigned int* err_word, cudaStream_t stream) {
+  return launch_fwd_any<false>(qp, kp, vp, row_ptr, col_idx, nullptr, kg, vg, order, BH, N, N, d,
+                               global_window, o, lse, err_word, stream);
+}
+
+cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp,
+                                 const int32_t* tile_ptr, const int32_t* tile_col,
+                                 const uint8_t* quarters, const void* kg, const void* vg,
+                                 int32_t* order, int BH, int N, int Ns, int d, int global_window,
+                                 void* o_s, float* lse_s, unsigned int* err_word,
+                                 cudaStream_t stream) {
+  return launch_fwd_any<true>(q_s, kp, vp, tile_ptr, tile_col, quarters, kg, vg, order, BH, N, Ns,
+                              d, global_window, o_s, lse_s, err_word, stream);
 }
 
 }  // namespace asa

@@ -8,6 +8,11 @@
 namespace asa {
 
 constexpr int kSamplesHost = 16;  // k: sampled tokens per block
+constexpr int kMaxBlocksHost = 2048;  // 262,144 tokens in blocks of 128
+
+// Device error word bit set when a caller-provided index (a CSR column, a pruning
+// source row or position) is out of range; the access is skipped.
+constexpr unsigned int kErrBadIndex = 32u;
 
 bool gilbert_order_host(int T, int Hg, int W, int32_t* out);
 
@@ -62,6 +67,36 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk,
                           void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream);
+
+// Exclusive scan of n int32 counts on one CTA: out[i] = sum_{k<i} in[k], out[n] and
+// *total (if non-null) = the sum.
+cudaError_t launch_scan(const int32_t* in, int n, int32_t* out, int32_t* total,
+                        cudaStream_t stream);
+
+// Query pruning with token filling (BSA).  q_s: [BH][Ns][d] bf16 compact queries,
+// `pack` blocks per 128-row tile; src_pos / src_row: [BH][N] int32.
+cudaError_t launch_prune(const void* qp, int BH, int N, int d, float r, int w, int pack, void* q_s,
+                         int Ns, int32_t* src_pos, int32_t* src_row, cudaStream_t stream);
+// Tile CSR (union of the tile's blocks' kept key blocks) with a quarter bit mask per
+// entry; counts: [BH * ntile] scratch.
+cudaError_t launch_prune_mask(const int32_t* row_ptr, const int32_t* col_idx, int BH, int nb,
+                              int pack, int32_t* counts, int32_t* tile_ptr, int32_t* tile_col,
+                              uint8_t* tile_quarters, int32_t* nnz_out, unsigned int* err_word,
+                              int num_sms, cudaStream_t stream);
+cudaError_t launch_fill_out(const void* o_s, const float* lse_s, const int32_t* src_row, int BH,
+                            int N, int Ns, int d, void* o, float* lse, unsigned int* err_word,
+                            int num_sms, cudaStream_t stream);
+cudaError_t launch_dout_fill(const void* dout, const float* lse, const int32_t* src_pos, int BH,
+                             int N, int d, void* dout2, float* lse2, unsigned int* err_word,
+                             int num_sms, cudaStream_t stream);
+// Forward over a packed tile CSR: q_s has Ns rows per head; quarters[e] says which
+// 32-row lane quarters of the tile see entry e; o_s, lse_s: [BH][Ns].
+cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp,
+                                 const int32_t* tile_ptr, const int32_t* tile_col,
+                                 const uint8_t* quarters, const void* kg, const void* vg,
+                                 int32_t* order, int BH, int N, int Ns, int d, int global_window,
+                                 void* o_s, float* lse_s, unsigned int* err_word,
+                                 cudaStream_t stream);
 
 // Failure-detection test hook: one bounded wait on a barrier nothing arrives at.
 cudaError_t launch_wait_timeout(unsigned int* err_word, long long limit, cudaStream_t stream);

@@ -266,6 +266,12 @@ cudaError_t csr_from_bitmap(const uint8_t* bitmap, int32_t* counts, int BH, int 
 
 }  // namespace
 
+cudaError_t launch_scan(const int32_t* in, int n, int32_t* out, int32_t* total,
+                        cudaStream_t stream) {
+  scan_kernel<<<1, 1024, 0, stream>>>(in, n, out, total);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_build_mask(const float* p_imp, int BH, int nb, float tau, uint8_t* bitmap,
                               int32_t* counts, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
                               int32_t* counts_t, int32_t* col_ptr_t, int32_t* row_idx_t, int num_sms,

@@ -1,0 +1,393 @@
+// Query pruning with token filling ("Bidirectional Sparse Attention for Faster Video
+// Diffusion Training", "Key designs", item 1), on ASA's blocks of 128 permuted tokens.
+//
+// A block is cut into windows of w consecutive tokens; the token in the middle of
+// each window (offset len/2) is its centre.  The block keeps every centre and the
+// other tokens with the largest 1 - cos(q_centre, q_i), K = max(ceil(r L), windows)
+// in all (ties to the lower position).  Kept queries are packed into a compact
+// buffer of 128-row tiles holding `pack` blocks each (slots of 128/pack rows, a
+// block's kept rows in position order, the rest of its slot zero), so that one
+// tcgen05 tile computes the kept rows of `pack` blocks at once.  The attention of a
+// tile runs over the union of its blocks' kept key blocks, and each key block of the
+// union carries a bit per 32-row TMEM lane quarter telling which rows may see it.
+// A pruned token then takes its centre's output row and LSE (token filling).
+#include "common.cuh"
+#include "internal.h"
+
+namespace asa {
+
+namespace {
+
+constexpr float kCosEps = 1e-8f;
+constexpr int kPackThreads = 256;  // 8 warps, one tile each
+constexpr int kMaxWords = kMaxBlocksHost / 32;
+
+template <int E>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float* x) {
+  if constexpr (E == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    x[0] = __uint_as_float(u.x << 16);
+    x[1] = __uint_as_float(u.x & 0xffff0000u);
+    x[2] = __uint_as_float(u.y << 16);
+    x[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    x[0] = __uint_as_float(u << 16);
+    x[1] = __uint_as_float(u & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One CTA per (b, h, block I); 128 threads.
+template <int D>
+__global__ void __launch_bounds__(128)
+    prune_kernel(const __nv_bfloat16* __restrict__ qp, int N, int nb, float r, int w, int pack,
+                 __nv_bfloat16* __restrict__ q_s, int Ns, int32_t* __restrict__ src_pos,
+                 int32_t* __restrict__ src_row) {
+  __shared__ float s_dis[kBlock];
+  __shared__ int s_slot[kBlock];
+  __shared__ int s_tok[kBlock];
+  __shared__ int s_wtot[4];
+  const int bh = blockIdx.x / nb, I = blockIdx.x % nb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int s0 = I * kBlock;
+  const int L = min(kBlock, N - s0);
+  const __nv_bfloat16* qb = qp + (static_cast<int64_t>(bh) * N + s0) * D;
+  auto centre = [&](int t) {
+    const int ws = (t / w) * w;
+    return ws + min(w, L - ws) / 2;
+  };
+
+  // 1 - cos(q_centre, q_t): one warp per token, D/32 elements per lane, fp32
+  constexpr int E = D / 32;
+  for (int t = warp; t < L; t += 4) {
+    const int c = centre(t);
+    float a[E], b[E];
+    load_bf16<E>(qb + static_cast<int64_t>(t) * D + lane * E, a);
+    load_bf16<E>(qb + static_cast<int64_t>(c) * D + lane * E, b);
+    float dot = 0.f, na = 0.f, nc = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      dot = fmaf(a[e], b[e], dot);
+      na = fmaf(a[e], a[e], na);
+      nc = fmaf(b[e], b[e], nc);
+    }
+    dot = warp_sum_f(dot);
+    na = warp_sum_f(na);
+    nc = warp_sum_f(nc);
+    const float den = fmaxf(sqrtf(na), kCosEps) * fmaxf(sqrtf(nc), kCosEps);
+    // centres are kept unconditionally: -inf keeps them out of the ranking
+    if (lane == 0) s_dis[t] = c == t ? -INFINITY : 1.f - dot / den;
+  }
+  __syncthreads();
+
+  // rank of each non-centre: tokens more dissimilar, or as dissimilar and earlier
+  const int windows = (L + w - 1) / w;
+  const int K = max(static_cast<int>(ceil(static_cast<double>(r) * L)), windows);
+  const int extra = K - windows;
+  bool kept = false;
+  if (tid < L) {
+    const float dt = s_dis[tid];
+    if (dt == -INFINITY) {
+      kept = true;
+    } else if (extra > 0) {
+      int rank = 0;
+      for (int u = 0; u < L; ++u) {
+        const float du = s_dis[u];
+        rank += (du > dt) | ((du == dt) & (u < tid));
+      }
+      kept = rank < extra;
+    }
+  }
+  // compact slots in position order
+  const unsigned bal = __ballot_sync(0xffffffffu, kept);
+  if (lane == 0) s_wtot[warp] = __popc(bal);
+  __syncthreads();
+  int base = 0;
+  for (int k = 0; k < warp; ++k) base += s_wtot[k];
+  const int nkept = s_wtot[0] + s_wtot[1] + s_wtot[2] + s_wtot[3];
+  const int slot = base + __popc(bal & ((1u << lane) - 1u));
+  s_slot[tid] = kept ? slot : -1;
+  if (kept) s_tok[slot] = tid;
+  __syncthreads();
+
+  const int S = kBlock / pack;
+  const int tile = I / pack, sub = I % pack;
+  const int row0 = tile * kBlock + sub * S;  // first compact row of this block
+  if (tid < L) {
+    const int c = kept ? tid : centre(tid);
+    const int64_t g = static_cast<int64_t>(bh) * N + s0 + tid;
+    src_pos[g] = s0 + c;
+    src_row[g] = row0 + s_slot[c];
+  }
+  // kept rows into their slots, zeros after them; the last block also zeroes the
+  // slots of its tile that no block owns
+  const int zero_end = (I == nb - 1) ? (tile + 1) * kBlock - row0 : S;
+  constexpr int kVec = D / 8;  // 16-byte pieces per row
+  __nv_bfloat16* qs = q_s + static_cast<int64_t>(bh) * Ns * D;
+  for (int sl = warp; sl < zero_end; sl += 4) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (lane < kVec) {
+      if (sl < nkept && sl < S)
+        v = reinterpret_cast<const uint4*>(qb + static_cast<int64_t>(s_tok[sl]) * D)[lane];
+      reinterpret_cast<uint4*>(qs + static_cast<int64_t>(row0 + sl) * D)[lane] = v;
+    }
+  }
+}
+
+// Kept key blocks of the tile's blocks as bitmaps in shared memory, one per slot.
+// Returns false if a column index is out of range (it is skipped).
+__device__ __forceinline__ bool tile_bitmaps(const int32_t* __restrict__ row_ptr,
+                                             const int32_t* __restrict__ col_idx, int r0,
+                                             int nsub, int nb, int words, uint32_t* bits,
+                                             int lane) {
+  for (int k = lane; k < 4 * words; k += 32) bits[k] = 0u;
+  __syncwarp();
+  bool ok = true;
+  for (int s = 0; s < nsub; ++s) {
+    const int e0 = row_ptr[r0 + s], e1 = row_ptr[r0 + s + 1];
+    for (int e = e0 + lane; e < e1; e += 32) {
+      const int J = col_idx[e];
+      if (J < 0 || J >= nb) {
+        ok = false;
+        continue;
+      }
+      atomicOr(&bits[s * words + (J >> 5)], 1u << (J & 31));
+    }
+  }
+  __syncwarp();
+  return ok;
+}
+
+__device__ __forceinline__ uint8_t slot_quarters(int s, int pack) {
+  const int q = 4 / pack;
+  return static_cast<uint8_t>(((1u << q) - 1u) << (s * q));
+}
+
+// counts[bh * ntile + t] = number of key blocks kept by any block of tile t
+__global__ void __launch_bounds__(kPackThreads)
+    pack_count_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                      int BH, int nb, int pack, int32_t* __restrict__ counts,
+                      unsigned int* __restrict__ err_word) {
+  __shared__ uint32_t sbits[kPackThreads / 32][4 * kMaxWords];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int ntile = (nb + pack - 1) / pack;
+  const int words = (nb + 31) / 32;
+  uint32_t* bits = sbits[wib];
+  for (int idx = blockIdx.x * (kPackThreads / 32) + wib; idx < BH * ntile;
+       idx += gridDim.x * (kPackThreads / 32)) {
+    const int bh = idx / ntile, t = idx % ntile;
+    const int nsub = min(pack, nb - t * pack);
+    const bool ok = tile_bitmaps(row_ptr, col_idx, bh * nb + t * pack, nsub, nb, words, bits, lane);
+    if (__any_sync(0xffffffffu, !ok) && lane == 0) atomicOr(err_word, kErrBadIndex);
+    int c = 0;
+    for (int k = lane; k < words; k += 32) {
+      uint32_t u = 0;
+      for (int s = 0; s < nsub; ++s) u |= bits[s * words + k];
+      c += __popc(u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) counts[idx] = c;
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kPackThreads)
+    pack_fill_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                     int BH, int nb, int pack, const int32_t* __restrict__ tile_ptr,
+                     int32_t* __restrict__ tile_col, uint8_t* __restrict__ tile_quarters) {
+  __shared__ uint32_t sbits[kPackThreads / 32][4 * kMaxWords];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int ntile = (nb + pack - 1) / pack;
+  const int words = (nb + 31) / 32;
+  uint32_t* bits = sbits[wib];
+  for (int idx = blockIdx.x * (kPackThreads / 32) + wib; idx < BH * ntile;
+       idx += gridDim.x * (kPackThreads / 32)) {
+    const int bh = idx / ntile, t = idx % ntile;
+    const int nsub = min(pack, nb - t * pack);
+    tile_bitmaps(row_ptr, col_idx, bh * nb + t * pack, nsub, nb, words, bits, lane);
+    int pos = tile_ptr[idx];
+    for (int k0 = 0; k0 < words; k0 += 32) {
+      const int k = k0 + lane;
+      uint32_t u = 0;
+      if (k < words)
+        for (int s = 0; s < nsub; ++s) u |= bits[s * words + k];
+      const int c = __popc(u);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int p = pos + incl - c;
+      while (u != 0u) {
+        const int b = __ffs(u) - 1;
+        u &= u - 1u;
+        uint8_t q = 0;
+        for (int s = 0; s < nsub; ++s)
+          if ((bits[s * words + k] >> b) & 1u) q |= slot_quarters(s, pack);
+        tile_col[p] = k * 32 + b;
+        tile_quarters[p] = q;
+        ++p;
+      }
+      pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+  }
+}
+
+// O[bh, i] = O_s[bh, src_row[i]], LSE likewise: D/8 threads per row, 16 bytes each
+template <int D>
+__global__ void __launch_bounds__(256)
+    fill_out_kernel(const __nv_bfloat16* __restrict__ o_s, const float* __restrict__ lse_s,
+                    const int32_t* __restrict__ src_row, int64_t rows, int N, int Ns,
+                    __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                    unsigned int* __restrict__ err_word) {
+  constexpr int kVec = D / 8;
+  const int64_t total = rows * kVec;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = g / kVec;
+    const int v = static_cast<int>(g - row * kVec);
+    const int64_t bh = row / N;
+    const int sr = src_row[row];
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    float l = -INFINITY;
+    if (sr >= 0 && sr < Ns) {
+      const int64_t srow = bh * Ns + sr;
+      x = reinterpret_cast<const uint4*>(o_s + srow * D)[v];
+      l = lse_s[srow];
+    } else if (v == 0) {
+      atomicOr(err_word, kErrBadIndex);
+    }
+    reinterpret_cast<uint4*>(o + row * D)[v] = x;
+    if (v == 0) lse[row] = l;
+  }
+}
+
+// Backward inputs under pruning: dO'[i] = sum of dO[j] over the tokens j of i's block
+// with src_pos[j] = i when token i is kept (src_pos[i] = i), else 0; lse'[i] = lse[i]
+// for kept rows, +inf for pruned ones (their probabilities vanish).  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256)
+    dout_fill_kernel(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                     const int32_t* __restrict__ src_pos, int64_t rows, int N,
+                     __nv_bfloat16* __restrict__ dout2, float* __restrict__ lse2,
+                     unsigned int* __restrict__ err_word) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < rows; row += warps) {
+    const int64_t bh = row / N;
+    const int i = static_cast<int>(row - bh * N);
+    const int s0 = (i / kBlock) * kBlock;
+    const int L = min(kBlock, N - s0);
+    const int32_t* sp = src_pos + bh * N;
+    const int p = sp[i];
+    bool bad = p < s0 || p >= s0 + L || sp[p] != p;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    if (!bad && p == i) {
+      for (int j0 = 0; j0 < L; j0 += 32) {
+        const int j = j0 + lane;
+        unsigned m = __ballot_sync(0xffffffffu, j < L && sp[s0 + j] == i);
+        while (m != 0u) {
+          const int b = __ffs(m) - 1;
+          m &= m - 1u;
+          float x[E];
+          load_bf16<E>(dout + (bh * N + s0 + j0 + b) * D + lane * E, x);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] += x[e];
+        }
+      }
+    }
+    __nv_bfloat16* dst = dout2 + row * D + lane * E;
+    if constexpr (E == 4) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0], acc[1]);
+    }
+    if (lane == 0) {
+      lse2[row] = (!bad && p == i) ? lse[row] : INFINITY;
+      if (bad) atomicOr(err_word, kErrBadIndex);
+    }
+  }
+}
+
+unsigned grid_of(int64_t work, int per_block, int num_sms, int per_sm) {
+  int64_t b = (work + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+  if (b > cap) b = cap;
+  if (b < 1) b = 1;
+  return static_cast<unsigned>(b);
+}
+
+}  // namespace
+
+cudaError_t launch_prune(const void* qp, int BH, int N, int d, float r, int w, int pack, void* q_s,
+                         int Ns, int32_t* src_pos, int32_t* src_row, cudaStream_t stream) {
+  const int nb = (N + kBlock - 1) / kBlock;
+  const auto* q = static_cast<const __nv_bfloat16*>(qp);
+  auto* qs = static_cast<__nv_bfloat16*>(q_s);
+  if (d == 128)
+    prune_kernel<128><<<BH * nb, 128, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos, src_row);
+  else
+    prune_kernel<64><<<BH * nb, 128, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos, src_row);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prune_mask(const int32_t* row_ptr, const int32_t* col_idx, int BH, int nb,
+                              int pack, int32_t* counts, int32_t* tile_ptr, int32_t* tile_col,
+                              uint8_t* tile_quarters, int32_t* nnz_out, unsigned int* err_word,
+                              int num_sms, cudaStream_t stream) {
+  const int ntile = (nb + pack - 1) / pack;
+  const int64_t tiles = static_cast<int64_t>(BH) * ntile;
+  const unsigned grid = grid_of(tiles, kPackThreads / 32, num_sms, 8);
+  pack_count_kernel<<<grid, kPackThreads, 0, stream>>>(row_ptr, col_idx, BH, nb, pack, counts,
+                                                        err_word);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_scan(counts, static_cast<int>(tiles), tile_ptr, nnz_out, stream);
+  if (e != cudaSuccess) return e;
+  pack_fill_kernel<<<grid, kPackThreads, 0, stream>>>(row_ptr, col_idx, BH, nb, pack, tile_ptr,
+                                                       tile_col, tile_quarters);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_out(const void* o_s, const float* lse_s, const int32_t* src_row, int BH,
+                            int N, int Ns, int d, void* o, float* lse, unsigned int* err_word,
+                            int num_sms, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(BH) * N;
+  const unsigned grid = grid_of(rows * (d / 8), 256, num_sms, 8);
+  const auto* src = static_cast<const __nv_bfloat16*>(o_s);
+  auto* dst = static_cast<__nv_bfloat16*>(o);
+  if (d == 128)
+    fill_out_kernel<128><<<grid, 256, 0, stream>>>(src, lse_s, src_row, rows, N, Ns, dst, lse, err_word);
+  else
+    fill_out_kernel<64><<<grid, 256, 0, stream>>>(src, lse_s, src_row, rows, N, Ns, dst, lse, err_word);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dout_fill(const void* dout, const float* lse, const int32_t* src_pos, int BH,
+                             int N, int d, void* dout2, float* lse2, unsigned int* err_word,
+                             int num_sms, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(BH) * N;
+  const unsigned grid = grid_of(rows, 8, num_sms, 8);
+  const auto* src = static_cast<const __nv_bfloat16*>(dout);
+  auto* dst = static_cast<__nv_bfloat16*>(dout2);
+  if (d == 128)
+    dout_fill_kernel<128><<<grid, 256, 0, stream>>>(src, lse, src_pos, rows, N, dst, lse2, err_word);
+  else
+    dout_fill_kernel<64><<<grid, 256, 0, stream>>>(src, lse, src_pos, rows, N, dst, lse2, err_word);
+  return cudaGetLastError();
+}
+
+}  // namespace asa
