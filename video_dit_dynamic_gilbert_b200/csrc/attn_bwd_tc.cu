@@ -986,8 +986,8 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
       e = cudaGetLastError();
     }
   }
-  if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, ws.ord_r, stream);
-  if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, ws.ord_c, stream);
+  if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, nb, ws.ord_r, stream);
+  if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, nb, ws.ord_c, stream);
   if (e != cudaSuccess) return e;
   if (d == 128)
     return launch_kernels<128>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ws, BH, N, G, gw,

@@ -464,24 +464,26 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
 // Launch order of the query blocks: heads in order (concurrent CTAs then share one
 // head's K and V in L2), and inside each head the query blocks with the most kept
 // blocks first, so that the grid ends on short CTAs.  One CTA per head: a counting
-// sort of its nb rows by kept-block count.
+// sort of its nrows rows by entry count (bins 0..maxc; a larger count, possible only
+// in a malformed CSR, is sorted as maxc).
 __global__ void __launch_bounds__(1024) lpt_order_kernel(const int32_t* __restrict__ row_ptr,
-                                                        int nb, int32_t* __restrict__ order) {
-  extern __shared__ int32_t start[];  // nb + 1 bins
+                                                        int nrows, int maxc,
+                                                        int32_t* __restrict__ order) {
+  extern __shared__ int32_t start[];  // maxc + 1 bins
   __shared__ int32_t chunk_tot[1024];
   const int tid = threadIdx.x;
-  const int r0 = blockIdx.x * nb;
-  for (int c = tid; c <= nb; c += blockDim.x) start[c] = 0;
+  const int r0 = blockIdx.x * nrows;
+  auto count = [&](int r) { return min(max(row_ptr[r0 + r + 1] - row_ptr[r0 + r], 0), maxc); };
+  for (int c = tid; c <= maxc; c += blockDim.x) start[c] = 0;
   __syncthreads();
-  for (int r = tid; r < nb; r += blockDim.x)
-    atomicAdd(&start[row_ptr[r0 + r + 1] - row_ptr[r0 + r]], 1);
+  for (int r = tid; r < nrows; r += blockDim.x) atomicAdd(&start[count(r)], 1);
   __syncthreads();
   // exclusive scan over bins in descending count: bin c starts after all bins > c
-  const int nbins = nb + 1;
+  const int nbins = maxc + 1;
   const int per = (nbins + blockDim.x - 1) / blockDim.x;
   const int lo = min(nbins, tid * per), hi = min(nbins, lo + per);  // reversed bin index
   int32_t sum = 0;
-  for (int k = lo; k < hi; ++k) sum += start[nb - k];
+  for (int k = lo; k < hi; ++k) sum += start[maxc - k];
   chunk_tot[tid] = sum;
   __syncthreads();
   if (tid == 0) {
@@ -495,15 +497,12 @@ __global__ void __launch_bounds__(1024) lpt_order_kernel(const int32_t* __restri
   __syncthreads();
   int32_t run = chunk_tot[tid];
   for (int k = lo; k < hi; ++k) {
-    const int32_t v = start[nb - k];
-    start[nb - k] = run;
+    const int32_t v = start[maxc - k];
+    start[maxc - k] = run;
     run += v;
   }
   __syncthreads();
-  for (int r = tid; r < nb; r += blockDim.x) {
-    const int c = row_ptr[r0 + r + 1] - row_ptr[r0 + r];
-    order[r0 + atomicAdd(&start[c], 1)] = r0 + r;
-  }
+  for (int r = tid; r < nrows; r += blockDim.x) order[r0 + atomicAdd(&start[count(r)], 1)] = r0 + r;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -549,9 +548,9 @@ bool make_map_rows_f16(CUtensorMap* m, const void* ptr, int BH, int rows, int D)
   return make_map_dtype(m, ptr, BH, rows, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
 
-cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
+cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nrows, int maxc, int32_t* order,
                              cudaStream_t stream) {
-  lpt_order_kernel<<<BH, 1024, (nb + 1) * sizeof(int32_t), stream>>>(ptr, nb, order);
+  lpt_order_kernel<<<BH, 1024, (maxc + 1) * sizeof(int32_t), stream>>>(ptr, nrows, maxc, order);
   return cudaGetLastError();
 }
 
@@ -580,7 +579,8 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   if (regs_checked < 0) return cudaErrorInvalidConfiguration;
   const long long limit = 1ll << 31;  // ~1 s of SM clock per wait
   const int rows = nb * BH;
-  e = launch_lpt_order(row_ptr, BH, nb, order, stream);
+  // a row holds at most one entry per key block
+  e = launch_lpt_order(row_ptr, BH, nb, (N + kBlock - 1) / kBlock, order, stream);
   if (e != cudaSuccess) return e;
   fwd_tc_kernel<D, NST, kPruned><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, quarters, order, N, Nq, nb,

@@ -53,9 +53,10 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
                           int BH, int N, int d, int global_window, void* o, float* lse,
                           unsigned int* err_word, cudaStream_t stream);
 
-// Launch order of the blocks of a CSR (ptr[BH * nb + 1], global offsets): heads in
-// order, inside each head the rows with the most entries first.
-cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nb, int32_t* order,
+// Launch order of the rows of a CSR (ptr[BH * nrows + 1], global offsets): heads in
+// order, inside each head the rows with the most entries first; maxc bounds a row's
+// entry count (the number of key blocks).
+cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nrows, int maxc, int32_t* order,
                              cudaStream_t stream);
 
 // Backward workspace (bytes, 256-aligned pieces): lse2 and D [BH][nb*128] f32,
