@@ -43,33 +43,51 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-// One CTA per (b, h, block I); 128 threads.
+constexpr int kPruneThreads = 256;
+constexpr int kPruneWarps = kPruneThreads / 32;
+
+// One CTA per (b, h, block I).  The block's queries are staged in shared memory with
+// independent 16-byte loads; each warp then takes tokens t = warp, warp + 8, ... and
+// reads rows t and centre(t) from shared memory (one contiguous row per warp access).
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kPruneThreads)
     prune_kernel(const __nv_bfloat16* __restrict__ qp, int N, int nb, float r, int w, int pack,
                  __nv_bfloat16* __restrict__ q_s, int Ns, int32_t* __restrict__ src_pos,
                  int32_t* __restrict__ src_row) {
+  __shared__ __align__(16) __nv_bfloat16 s_q[kBlock * D];
   __shared__ float s_dis[kBlock];
   __shared__ int s_slot[kBlock];
   __shared__ int s_tok[kBlock];
-  __shared__ int s_wtot[4];
+  __shared__ int s_wtot[kPruneWarps];
   const int bh = blockIdx.x / nb, I = blockIdx.x % nb;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s0 = I * kBlock;
   const int L = min(kBlock, N - s0);
   const __nv_bfloat16* qb = qp + (static_cast<int64_t>(bh) * N + s0) * D;
+  constexpr int kVec = D / 8;  // 16-byte pieces per row
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(qb);
+    uint4* dst = reinterpret_cast<uint4*>(s_q);
+    for (int i = tid; i < L * kVec; i += kPruneThreads) dst[i] = src[i];
+  }
+  __syncthreads();
   auto centre = [&](int t) {
     const int ws = (t / w) * w;
     return ws + min(w, L - ws) / 2;
   };
 
-  // 1 - cos(q_centre, q_t): one warp per token, D/32 elements per lane, fp32
+  // 1 - cos(q_centre, q_t) in fp32, D/32 elements per lane; centres are kept
+  // unconditionally: -inf keeps them out of the ranking
   constexpr int E = D / 32;
-  for (int t = warp; t < L; t += 4) {
+  for (int t = warp; t < L; t += kPruneWarps) {
     const int c = centre(t);
+    if (c == t) {
+      if (lane == 0) s_dis[t] = -INFINITY;
+      continue;
+    }
     float a[E], b[E];
-    load_bf16<E>(qb + static_cast<int64_t>(t) * D + lane * E, a);
-    load_bf16<E>(qb + static_cast<int64_t>(c) * D + lane * E, b);
+    load_bf16<E>(s_q + t * D + lane * E, a);
+    load_bf16<E>(s_q + c * D + lane * E, b);
     float dot = 0.f, na = 0.f, nc = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -81,8 +99,7 @@ __global__ void __launch_bounds__(128)
     na = warp_sum_f(na);
     nc = warp_sum_f(nc);
     const float den = fmaxf(sqrtf(na), kCosEps) * fmaxf(sqrtf(nc), kCosEps);
-    // centres are kept unconditionally: -inf keeps them out of the ranking
-    if (lane == 0) s_dis[t] = c == t ? -INFINITY : 1.f - dot / den;
+    if (lane == 0) s_dis[t] = 1.f - dot / den;
   }
   __syncthreads();
 
@@ -108,11 +125,14 @@ __global__ void __launch_bounds__(128)
   const unsigned bal = __ballot_sync(0xffffffffu, kept);
   if (lane == 0) s_wtot[warp] = __popc(bal);
   __syncthreads();
-  int base = 0;
-  for (int k = 0; k < warp; ++k) base += s_wtot[k];
-  const int nkept = s_wtot[0] + s_wtot[1] + s_wtot[2] + s_wtot[3];
+  int base = 0, nkept = 0;
+#pragma unroll
+  for (int k = 0; k < kPruneWarps; ++k) {
+    base += k < warp ? s_wtot[k] : 0;
+    nkept += s_wtot[k];
+  }
   const int slot = base + __popc(bal & ((1u << lane) - 1u));
-  s_slot[tid] = kept ? slot : -1;
+  if (tid < kBlock) s_slot[tid] = kept ? slot : -1;
   if (kept) s_tok[slot] = tid;
   __syncthreads();
 
@@ -126,17 +146,15 @@ __global__ void __launch_bounds__(128)
     src_row[g] = row0 + s_slot[c];
   }
   // kept rows into their slots, zeros after them; the last block also zeroes the
-  // slots of its tile that no block owns
+  // slots of its tile that no block owns.  16-byte pieces, kVec per row.
   const int zero_end = (I == nb - 1) ? (tile + 1) * kBlock - row0 : S;
-  constexpr int kVec = D / 8;  // 16-byte pieces per row
-  __nv_bfloat16* qs = q_s + static_cast<int64_t>(bh) * Ns * D;
-  for (int sl = warp; sl < zero_end; sl += 4) {
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (lane < kVec) {
-      if (sl < nkept && sl < S)
-        v = reinterpret_cast<const uint4*>(qb + static_cast<int64_t>(s_tok[sl]) * D)[lane];
-      reinterpret_cast<uint4*>(qs + static_cast<int64_t>(row0 + sl) * D)[lane] = v;
-    }
+  uint4* qs = reinterpret_cast<uint4*>(q_s + (static_cast<int64_t>(bh) * Ns + row0) * D);
+  const uint4* sq = reinterpret_cast<const uint4*>(s_q);
+  for (int i = tid; i < zero_end * kVec; i += kPruneThreads) {
+    const int sl = i / kVec, v = i - sl * kVec;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (sl < nkept && sl < S) x = sq[s_tok[sl] * kVec + v];
+    qs[i] = x;
   }
 }
 
@@ -338,9 +356,11 @@ cudaError_t launch_prune(const void* qp, int BH, int N, int d, float r, int w, i
   const auto* q = static_cast<const __nv_bfloat16*>(qp);
   auto* qs = static_cast<__nv_bfloat16*>(q_s);
   if (d == 128)
-    prune_kernel<128><<<BH * nb, 128, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos, src_row);
+    prune_kernel<128><<<BH * nb, kPruneThreads, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos,
+                                                              src_row);
   else
-    prune_kernel<64><<<BH * nb, 128, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos, src_row);
+    prune_kernel<64><<<BH * nb, kPruneThreads, 0, stream>>>(q, N, nb, r, w, pack, qs, Ns, src_pos,
+                                                             src_row);
   return cudaGetLastError();
 }
 
