@@ -653,6 +653,10 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
     pfwd_ms = timeit(lambda: asa.asa_sparse_attn_fwd_pruned(pr, kp, vp, ptm, workspace=pws,
                                                              out=po, lse=plse))
     fwd_ms = timeit(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, tmask))
+    pbws = asa.bwd_pruned_workspace(B, H, N, d, pr.pack, dev)
+    pgrads = tuple(torch.empty_like(qp) for _ in range(3))
+    pbwd_ms = timeit(lambda: asa.asa_sparse_attn_bwd_pruned(pr, kp, vp, dout, plse, ptm,
+                                                            workspace=pbws, outs=pgrads), reps=5)
     pflops, nkept = _pruned_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
                                   pr.src_pos.cpu().numpy(), B, H, N, d)
     union = int(ptm.nnz.item())
@@ -664,6 +668,8 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
             "prune_ms": prune_ms, "prune_mask_ms": pmask_ms, "fwd_ms": pfwd_ms,
             "fwd_effective_tflops": pflops / pfwd_ms / 1e9,
             "unpruned_fwd_ms": fwd_ms,
+            "bwd_ms": pbwd_ms, "unpruned_bwd_ms": bwd_ms,
+            "bwd_effective_tflops": 2.5 * pflops / pbwd_ms / 1e9,
             "speedup_total": fwd_ms / (prune_ms + pmask_ms + pfwd_ms),
         },
         "dense_ours_fwd_ms": ours_dense, "dense_ours_tflops": dense_flops / ours_dense / 1e9,

@@ -309,26 +309,32 @@ int asa_sparse_attn_fwd_pruned(const void* q_s, const void* kp, const void* vp,
                                void* workspace, size_t ws_bytes, void* o, float* lse,
                                void* stream);
 
-/* Workspace bytes of asa_sparse_attn_bwd_pruned: asa_bwd_workspace_size plus the
- * gathered output gradient (bf16 [B, H, N, d]) and the row LSEs (fp32 [B, H, N]). */
-size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int global_window);
+/* Workspace bytes of asa_sparse_attn_bwd_pruned: the backward's pieces with the query
+ * side in the compact layout (lse2, D, fp16 queries: B*H*Ns rows), the compact output
+ * gradient and dQ (bf16 [B, H, Ns, d] each), and the transposed tile CSR (a dense
+ * [B*H][Ns/128][ceil(N/128)] byte matrix, its counts, pointers, tile indices and
+ * quarter bits).  0 for invalid sizes. */
+size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int pack, int global_window);
 
 /*
- * Backward with query pruning under the fixed mask: with dO'[c] = the sum of dO[i]
- * over the tokens i with src_pos[i] = c (stored in bf16; zero on pruned rows) it
- * computes asa_sparse_attn_bwd's gradients for the kept rows, and pruned rows get
- * dQ = 0 (their LSE is taken as +inf, so their probabilities vanish).  Inputs as in
- * asa_sparse_attn_bwd, with lse the pruned forward's and src_pos from
- * asa_prune_queries (each token must map to a token of its own block that maps to
- * itself; other rows are zeroed and reported as ASA_ERR_INVALID_ARG).  The kept
- * rows run in the full layout: the backward does the unpruned amount of work.
+ * Backward with query pruning under the fixed mask, on the packed tiles of the pruned
+ * forward.  A pruned token's output is its centre's row, so with dO'[c] = the sum of
+ * dO[i] over the tokens i with src_pos[i] = c (stored in bf16) it computes
+ * asa_sparse_attn_bwd's gradients of the kept rows only, and pruned rows get dQ = 0.
+ * The query side runs over q_s's compact rows (a (tile, key block) entry restricted to
+ * the lane quarters of tile_quarters); the key side walks the transposed tile CSR,
+ * built in the workspace.  Inputs: q_s, src_pos, src_row from asa_prune_queries
+ * (each token must map to a kept token of its own block; other rows are skipped and
+ * reported as ASA_ERR_INVALID_ARG), tile_* from asa_prune_mask, lse from
+ * asa_sparse_attn_fwd_pruned, dout bf16 [B, H, N, d] (permuted layout), kp, vp as in
+ * the forward.  Outputs dq, dk, dv bf16 [B, H, N, d].  Deterministic.
  */
-int asa_sparse_attn_bwd_pruned(const void* qp, const void* kp, const void* vp, const void* dout,
-                               const float* lse, const int32_t* src_pos, const int32_t* row_ptr,
-                               const int32_t* col_idx, const int32_t* col_ptr_t,
-                               const int32_t* row_idx_t, int B, int H, int N, int d, int block,
-                               int global_window, void* workspace, size_t ws_bytes, void* dq,
-                               void* dk, void* dv, void* stream);
+int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, const void* dout,
+                               const float* lse, const int32_t* src_pos, const int32_t* src_row,
+                               const int32_t* tile_ptr, const int32_t* tile_col,
+                               const uint8_t* tile_quarters, int B, int H, int N, int d, int block,
+                               int pack, int global_window, void* workspace, size_t ws_bytes,
+                               void* dq, void* dk, void* dv, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of

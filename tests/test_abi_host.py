@@ -201,9 +201,15 @@ def test_prune_rejects(L):
     fwd[12] = 2
     fwd[13] = -1     # global_window
     assert L.asa_sparse_attn_fwd_pruned(*fwd) == asa.ASA_ERR_INVALID_ARG
-    bwd = [FAKE] * 10 + [1, 2, 1024, 64, 128, 0, None, 0] + [FAKE] * 3 + [None]
+    bwd = [FAKE] * 10 + [1, 2, 1024, 64, 128, 2, 0, None, 0] + [FAKE] * 3 + [None]
     assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_WORKSPACE
+    bwd[15] = 3      # pack
+    assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_INVALID_ARG
+    bwd[15] = 2
     bwd[5] = None    # src_pos
+    assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_INVALID_ARG
+    bwd[5] = FAKE
+    bwd[9] = None    # tile_quarters
     assert L.asa_sparse_attn_bwd_pruned(*bwd) == asa.ASA_ERR_INVALID_ARG
 
 
@@ -216,6 +222,11 @@ def test_prune_workspace_sizes(L):
     assert fw >= tiles * 4 + tiles * 128 * (d * 2 + 4)      # order, compact O and LSE
     G = -(-N // 64)
     assert L.asa_fwd_pruned_workspace_size(1, 12, N, d, 2, 64) - fw >= 2 * BH * G * d * 2
-    bw = L.asa_bwd_pruned_workspace_size(1, 12, N, d, 0)
-    assert bw >= L.asa_bwd_workspace_size(1, 12, N, d, 0) + BH * N * (d * 2 + 4)
-    assert L.asa_bwd_pruned_workspace_size(1, 12, N, 96, 0) == 0
+    # the packed backward: query side over 2 x 128 compact rows per tile, the compact
+    # dO' and dQ, the dense quarter matrix and the transposed tile CSR
+    Ns = 128 * 128
+    bw = L.asa_bwd_pruned_workspace_size(1, 12, N, d, 2, 0)
+    assert bw >= BH * Ns * (2 * 4 + 2 * d * 2) + BH * N * d * 2 + BH * 128 * 256 * 6
+    assert bw < L.asa_bwd_workspace_size(1, 12, N, d, 0) + BH * Ns * d * 4 + BH * 128 * 256 * 8
+    assert L.asa_bwd_pruned_workspace_size(1, 12, N, 96, 2, 0) == 0
+    assert L.asa_bwd_pruned_workspace_size(1, 12, N, d, 3, 0) == 0

@@ -161,13 +161,15 @@ def _expected_rows(O_full, L_full, src_or, sp_gpu, marg, centres):
     return O, L
 
 
-def _run_pruned_forward(name, r, w, gw=0, pack=0):
+def _run_pruned_forward(name, r, w, gw=0, pack=0, with_tiles=False):
     wl, x, perm, ref, mask, dev = setup_case(name)
     pr = asa.asa_prune_queries(dev["q"], r, w, pack=pack)
     bm = upload_mask(mask, wl.N)
     tm = asa.asa_prune_mask(bm, pr.pack)
     o, lse = asa.asa_sparse_attn_fwd_pruned(pr, dev["k"], dev["v"], tm, global_window=gw)
     asa.asa_check_device_status()
+    if with_tiles:
+        return wl, ref, mask, dev, pr, bm, tm, o, lse
     return wl, ref, mask, dev, pr, bm, o, lse
 
 
@@ -207,17 +209,22 @@ def test_forward_keep_all_equals_unpruned():
     assert torch.equal(lse, lse_std)
 
 
-@pytest.mark.parametrize("name,r,w,gw", [("tiny", 0.5, 8, 0), ("one-ragged-block", 0.5, 8, 0),
-                                         ("d128-ragged", 0.3, 8, 0), ("d64-b2", 0.5, 8, 64)])
-def test_backward_pruned_matches_oracle(name, r, w, gw):
-    wl, ref, mask, dev, pr, bm, o, lse = _run_pruned_forward(name, r, w, gw)
+@pytest.mark.parametrize("name,r,w,gw,pack", [("tiny", 0.5, 8, 0, 0), ("one-ragged-block", 0.5, 8, 0, 0),
+                                              ("d128-ragged", 0.3, 8, 0, 0), ("d64-b2", 0.5, 8, 64, 0),
+                                              ("multi-tile", 0.2, 8, 0, 4), ("multi-tile", 0.5, 8, 16, 0),
+                                              ("d128-ragged", 0.5, 8, 0, 1), ("d64-b2", 1.0, 8, 0, 1)])
+def test_backward_pruned_matches_oracle(name, r, w, gw, pack):
+    """Packed backward (pack 1, 2, 4; ASA and ASA_G) against the oracle's pruned
+    backward; pruned rows get dQ = 0 exactly."""
+    wl, ref, mask, dev, pr, bm, tm, o, lse = _run_pruned_forward(name, r, w, gw, pack=pack,
+                                                                 with_tiles=True)
     kept, src, dis = oracle.prune_queries(ref["q"], r, w)
     assert not oracle.marginal_tokens(kept, dis, w).any(), "seeded case has a near-tie"
     # a centre collects up to w output gradients: scale dO by 1/8 (exact) on both sides
     dout = ref["dout"] / 8
     dop = torch.from_numpy(dout).to(torch.bfloat16).cuda()
-    got = [f64(t) for t in asa.asa_sparse_attn_bwd_pruned(dev["q"], dev["k"], dev["v"], dop, lse,
-                                                            bm, pr, global_window=gw)]
+    got = [f64(t) for t in asa.asa_sparse_attn_bwd_pruned(pr, dev["k"], dev["v"], dop, lse, tm,
+                                                            global_window=gw)]
     asa.asa_check_device_status()
     dq_d, dkv_d = oracle.asa_backward_pruned(ref["q"], ref["k"], ref["v"], dout, mask, src,
                                              global_window=gw)
@@ -305,8 +312,23 @@ def test_bad_indices_are_reported():
     # a src_pos pointing outside its block
     bad2 = asa.QueryPrune(pr.q_s, pr.src_pos.clone(), pr.src_row, pr.pack, pr.r, pr.window, pr.N)
     bad2.src_pos[0, 0, 3] = 700
-    asa.asa_sparse_attn_bwd_pruned(dev["q"], dev["k"], dev["v"], dev["dout"], lse, bm, bad2)
+    asa.asa_sparse_attn_bwd_pruned(bad2, dev["k"], dev["v"], dev["dout"], lse, tm)
     with pytest.raises(asa.AsaError) as e:
         asa.asa_check_device_status()
     assert e.value.code == asa.ASA_ERR_INVALID_ARG
     asa.asa_check_device_status()
+
+
+@pytest.mark.parametrize("name", ["d64-b2", "d128-ragged"])
+def test_backward_keep_all_equals_unpruned(name):
+    """r = 1 keeps every query: the compact layout is the permuted one, every quarter
+    bit is set and the transposed tile CSR lists the same query blocks in the same
+    order, so the packed backward computes exactly the unpruned backward."""
+    wl, ref, mask, dev, pr, bm, tm, o, lse = _run_pruned_forward(name, 1.0, 8, with_tiles=True)
+    assert pr.pack == 1
+    got = asa.asa_sparse_attn_bwd_pruned(pr, dev["k"], dev["v"], dev["dout"], lse, tm)
+    o_std, lse_std = asa.asa_sparse_attn_fwd(dev["q"], dev["k"], dev["v"], bm)
+    std = asa.asa_sparse_attn_bwd(dev["q"], dev["k"], dev["v"], o_std, dev["dout"], lse_std, bm)
+    asa.asa_check_device_status()
+    for g, e, nm in zip(got, std, ("dQ", "dK", "dV")):
+        assert torch.equal(g.view(torch.int16), e.view(torch.int16)), nm

@@ -51,8 +51,8 @@ _SIGNATURES = {
     "asa_prune_mask": ([_vp, _vp] + [_c_int] * 4 + [_vp, _c_size] + [_vp] * 5, _c_int),
     "asa_fwd_pruned_workspace_size": ([_c_int] * 6, _c_size),
     "asa_sparse_attn_fwd_pruned": ([_vp] * 7 + [_c_int] * 7 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
-    "asa_bwd_pruned_workspace_size": ([_c_int] * 5, _c_size),
-    "asa_sparse_attn_bwd_pruned": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
+    "asa_bwd_pruned_workspace_size": ([_c_int] * 6, _c_size),
+    "asa_sparse_attn_bwd_pruned": ([_vp] * 10 + [_c_int] * 7 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),
@@ -435,28 +435,27 @@ def asa_sparse_attn_fwd_pruned(prune: QueryPrune, kp, vp, tmask: TileMask, globa
     return out, lse
 
 
-def bwd_pruned_workspace(B, H, N, d, device, global_window: int = 0):
-    return _workspace(lib().asa_bwd_pruned_workspace_size(B, H, N, d, global_window), device)
+def bwd_pruned_workspace(B, H, N, d, pack, device, global_window: int = 0):
+    return _workspace(lib().asa_bwd_pruned_workspace_size(B, H, N, d, pack, global_window), device)
 
 
-def asa_sparse_attn_bwd_pruned(qp, kp, vp, dout, lse, mask: BlockMask, prune: QueryPrune,
+def asa_sparse_attn_bwd_pruned(prune: QueryPrune, kp, vp, dout, lse, tmask: TileMask,
                                global_window: int = 0, workspace=None, outs=None, stream=None):
-    """dQ, dK, dV [B, H, N, d] bf16 with query pruning under the fixed mask: pruned
-    tokens' output gradients go to their centres; pruned rows get dQ = 0."""
-    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp), ("dout", dout)):
+    """dQ, dK, dV [B, H, N, d] bf16 with query pruning under the fixed mask, on the
+    pruned forward's packed tiles: pruned tokens' output gradients go to their
+    centres; pruned rows get dQ = 0."""
+    for n_, t in (("kp", kp), ("vp", vp), ("dout", dout)):
         _bf16_cuda(n_, t)
-    if mask.col_ptr_t is None:
-        raise ValueError("the backward needs the transposed CSR (transposed=True)")
-    B, H, N, d = qp.shape
+    B, H, N, d = kp.shape
     if workspace is None:
-        workspace = bwd_pruned_workspace(B, H, N, d, qp.device, global_window)
+        workspace = bwd_pruned_workspace(B, H, N, d, prune.pack, kp.device, global_window)
     if outs is None:
-        outs = tuple(torch.empty_like(qp) for _ in range(3))
+        outs = tuple(torch.empty_like(kp) for _ in range(3))
     _check(lib().asa_sparse_attn_bwd_pruned(
-        _ptr(qp), _ptr(kp), _ptr(vp), _ptr(dout), _ptr(lse), _ptr(prune.src_pos),
-        _ptr(mask.row_ptr), _ptr(mask.col_idx), _ptr(mask.col_ptr_t), _ptr(mask.row_idx_t),
-        B, H, N, d, BLOCK, global_window, _ptr(workspace), _ws_bytes(workspace),
-        *(_ptr(t) for t in outs), _stream(stream)))
+        _ptr(prune.q_s), _ptr(kp), _ptr(vp), _ptr(dout), _ptr(lse), _ptr(prune.src_pos),
+        _ptr(prune.src_row), _ptr(tmask.tile_ptr), _ptr(tmask.tile_col),
+        _ptr(tmask.tile_quarters), B, H, N, d, BLOCK, prune.pack, global_window, _ptr(workspace),
+        _ws_bytes(workspace), *(_ptr(t) for t in outs), _stream(stream)))
     return outs
 
 
@@ -514,6 +513,7 @@ class ASAAttention(torch.autograd.Function):
             op, lse = asa_sparse_attn_fwd_pruned(prune, kp, vp, tmask, global_window=global_window)
         ctx.save_for_backward(qp, kp, vp, op, lse)
         ctx.mask, ctx.grid, ctx.global_window, ctx.prune = mask, (T, Hg, W), global_window, prune
+        ctx.tmask = tmask if prune is not None else None
         return asa_unpermute(op, T, Hg, W)
 
     @staticmethod
@@ -525,7 +525,7 @@ class ASAAttention(torch.autograd.Function):
             grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
                                         global_window=ctx.global_window)
         else:
-            grads = asa_sparse_attn_bwd_pruned(qp, kp, vp, dop, lse, ctx.mask, ctx.prune,
+            grads = asa_sparse_attn_bwd_pruned(ctx.prune, kp, vp, dop, lse, ctx.tmask,
                                                global_window=ctx.global_window)
         dq, dk, dv = (asa_unpermute(g, T, Hg, W) for g in grads)
         return dq, dk, dv, None, None, None, None, None, None, None

@@ -625,48 +625,43 @@ int asa_sparse_attn_fwd_pruned(const void* q_s, const void* kp, const void* vp,
   return ASA_OK;
 }
 
-size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int global_window) {
-  const size_t base = asa_bwd_workspace_size(B, H, N, d, global_window);
-  if (base == 0) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  return align256(base) + align256(rows * d * 2) + align256(rows * sizeof(float));
+size_t asa_bwd_pruned_workspace_size(int B, int H, int N, int d, int pack, int global_window) {
+  if (B < 1 || H < 1 || N < 1 || N > ASA_MAX_TOKENS || (d != 64 && d != 128) ||
+      (pack != 1 && pack != 2 && pack != 4) || global_window < 0)
+    return 0;
+  const int Ns = asa_prune_rows(N, pack);
+  return asa::bwd_tc_pruned_workspace_bytes(B * H, N, Ns, d, global_window);
 }
 
-int asa_sparse_attn_bwd_pruned(const void* qp, const void* kp, const void* vp, const void* dout,
-                               const float* lse, const int32_t* src_pos, const int32_t* row_ptr,
-                               const int32_t* col_idx, const int32_t* col_ptr_t,
-                               const int32_t* row_idx_t, int B, int H, int N, int d, int block,
-                               int global_window, void* workspace, size_t ws_bytes, void* dq,
-                               void* dk, void* dv, void* stream) {
+int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, const void* dout,
+                               const float* lse, const int32_t* src_pos, const int32_t* src_row,
+                               const int32_t* tile_ptr, const int32_t* tile_col,
+                               const uint8_t* tile_quarters, int B, int H, int N, int d, int block,
+                               int pack, int global_window, void* workspace, size_t ws_bytes,
+                               void* dq, void* dk, void* dv, void* stream) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_block(block, ASA_SAMPLES));
-  const void* bf[] = {qp, kp, vp, dout, dq, dk, dv};
-  const char* names[] = {"qp", "kp", "vp", "dout", "dq", "dk", "dv"};
+  ASA_TRY(check_pack(pack));
+  const void* bf[] = {q_s, kp, vp, dout, dq, dk, dv};
+  const char* names[] = {"q_s", "kp", "vp", "dout", "dq", "dk", "dv"};
   for (int k = 0; k < 7; ++k) ASA_TRY(check_ptr(bf[k], names[k]));
   ASA_TRY(check_ptr(lse, "lse", false));
   ASA_TRY(check_ptr(src_pos, "src_pos", false));
-  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
-  ASA_TRY(check_ptr(col_idx, "col_idx", false));
-  ASA_TRY(check_ptr(col_ptr_t, "col_ptr_t", false));
-  ASA_TRY(check_ptr(row_idx_t, "row_idx_t", false));
+  ASA_TRY(check_ptr(src_row, "src_row", false));
+  ASA_TRY(check_ptr(tile_ptr, "tile_ptr", false));
+  ASA_TRY(check_ptr(tile_col, "tile_col", false));
+  if (tile_quarters == nullptr) return fail(ASA_ERR_INVALID_ARG, "tile_quarters is NULL");
   if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
-  ASA_TRY(check_ws(workspace, ws_bytes, asa_bwd_pruned_workspace_size(B, H, N, d, global_window)));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  char* p = static_cast<char*>(workspace);
-  void* bwd_ws = p;
-  p += align256(asa_bwd_workspace_size(B, H, N, d, global_window));
-  void* dout2 = p;
-  p += align256(rows * d * 2);
-  float* lse2 = reinterpret_cast<float*>(p);
+  ASA_TRY(check_ws(workspace, ws_bytes,
+                   asa_bwd_pruned_workspace_size(B, H, N, d, pack, global_window)));
   unsigned int* err_word = nullptr;
   cudaError_t e = device_error_word(&err_word);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
-  e = asa::launch_dout_fill(dout, lse, src_pos, B * H, N, d, dout2, lse2, err_word, num_sms_current(), s);
-  if (e != cudaSuccess) return cuda_fail(e, "gradient fill launch");
-  e = asa::launch_bwd_tc(qp, kp, vp, dout2, lse2, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
-                         d, global_window, bwd_ws, dq, dk, dv, err_word, num_sms_current(), s);
-  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  const int Ns = asa_prune_rows(N, pack);
+  e = asa::launch_bwd_tc_pruned(q_s, kp, vp, dout, lse, src_pos, src_row, tile_ptr, tile_col,
+                                tile_quarters, B * H, N, Ns, d, global_window, workspace, dq, dk,
+                                dv, err_word, num_sms_current(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pruned backward launch");
   return ASA_OK;
 }
 

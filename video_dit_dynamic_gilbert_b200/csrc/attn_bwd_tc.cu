@@ -233,7 +233,9 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 
 // ------------------------------------------------------------------ query-block kernel
 
-template <int D, bool kDPass>
+// kPruned: packed query tiles of the pruned forward; entry t is seen only by the lane
+// quarters whose bit is set in quarters[rbeg + t] (the others give it probability 0).
+template <int D, bool kDPass, bool kPruned>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_row_kernel(const __grid_constant__ CUtensorMap tmQ16,
                    const __grid_constant__ CUtensorMap tmdO,
@@ -241,10 +243,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmKg16,
                    const __grid_constant__ CUtensorMap tmVg, const int32_t* __restrict__ row_ptr,
-                   const int32_t* __restrict__ col_idx, const int32_t* __restrict__ order, int N,
-                   int nb, int Np, int G, float gbias2, float c2, float scale,
-                   const float* __restrict__ lse2, float* __restrict__ Dvec,
-                   __nv_bfloat16* __restrict__ dq,
+                   const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ quarters,
+                   const int32_t* __restrict__ order, int N, int Nq, int nb, int Np, int G,
+                   float gbias2, float c2, float scale, const float* __restrict__ lse2,
+                   float* __restrict__ Dvec, __nv_bfloat16* __restrict__ dq,
                    unsigned int* __restrict__ err_word, long long wait_limit) {
   using L = BwdLayout<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -372,6 +374,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const int64_t vrow = static_cast<int64_t>(bh) * Np + q0 + row;
     const float nl2 = -lse2[vrow];  // rows past N: -inf, so P = 0
+    const uint8_t* qbits = kPruned ? quarters + rbeg : nullptr;
     const float dd = kDPass ? 0.f : Dvec[vrow];
     auto wait_warp = [&](uint32_t bar, uint32_t parity) {
       const bool ok = tc::mbar_wait(bar, parity, wait_limit);
@@ -392,9 +395,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::tmem_wait_ld_dep32(s + 32);
       if (kDPass) warp_arrive(br.ds_full(t & 1), lane);
       float p[64];
-      // global tokens carry + ln(n) (log2(n) in these units)
+      // global tokens carry + ln(n) (log2(n) in these units); with query pruning a
+      // warp whose rows do not keep key block cols[t] gives it probability 0
       const bool glob = t >= nfine;
-      const float off = nl2 + (glob ? gbias2 : 0.f);
+      const bool mine = !kPruned || glob || ((qbits[t] >> quarter) & 1u);
+      const float off = mine ? nl2 + (glob ? gbias2 : 0.f) : -INFINITY;
       exp2_64(s, c2, [&](int) { return off; }, p);
       // key columns past N (the ragged last block) or past G get no weight
       const int nvalid = (glob ? min(kBlock, G - (t - nfine) * kBlock)
@@ -442,7 +447,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::named_bar_sync(1, 256);
       if (w == 1) red[row] = part;
       tc::named_bar_sync(1, 256);
-      if (w == 0 && q < N) Dvec[vrow] = part + red[row];
+      if (w == 0 && q < Nq) Dvec[vrow] = part + red[row];
     } else {
       bool have = n > 0 && !failed;
       if (have) {
@@ -454,7 +459,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       // warpgroup w writes columns [D/2 w, D/2 w + D/2) of its rows
-      __nv_bfloat16* drow = dq + (static_cast<int64_t>(bh) * N + (q < N ? q : 0)) * D + (D / 2) * w;
+      __nv_bfloat16* drow = dq + (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t a[32];
@@ -464,7 +469,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) a[k] = 0u;
         }
-        if (q < N) store_row_bf16(drow + 32 * c, a, scale);
+        if (q < Nq) store_row_bf16(drow + 32 * c, a, scale);
       }
     }
   }
@@ -494,8 +499,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ16,
                    const __grid_constant__ CUtensorMap tmdO, const int32_t* __restrict__ col_ptr_t,
-                   const int32_t* __restrict__ row_idx_t, const int32_t* __restrict__ order,
-                   int N, int nb, int Np, int G, int gw, float gbias2, float c2, float scale,
+                   const int32_t* __restrict__ row_idx_t, const uint8_t* __restrict__ tquarters,
+                   const int32_t* __restrict__ order, int N, int nbk, int nbq, int Np, int G,
+                   int gw, float gbias2, float c2, float scale,
                    const float* __restrict__ lse2, const float* __restrict__ Dvec,
                    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                    float* __restrict__ dKg32, float* __restrict__ dVg32,
@@ -509,20 +515,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int bh, k0, n;
   const int32_t* rows;
+  const uint8_t* tq = nullptr;        // quarter bits of the query tiles (query pruning)
   if constexpr (kGlobal) {
     const int ng = (G + kBlock - 1) / kBlock;
     bh = blockIdx.x / ng;
     k0 = (blockIdx.x % ng) * kBlock;  // first global token of the tile
-    n = nb;
+    n = nbq;
     rows = nullptr;                   // query block t at step t
   } else {
     const int colid = order[blockIdx.x];
-    const int J = colid % nb;
-    bh = colid / nb;
+    const int J = colid % nbk;
+    bh = colid / nbk;
     k0 = J * kBlock;
-    const int cbeg = col_ptr_t[bh * nb + J];
-    n = col_ptr_t[bh * nb + J + 1] - cbeg;
+    const int cbeg = col_ptr_t[bh * nbk + J];
+    n = col_ptr_t[bh * nbk + J + 1] - cbeg;
     rows = row_idx_t + cbeg;
+    if (tquarters != nullptr) tq = tquarters + cbeg;
   }
 
   const Bars br{base + L::kBars};
@@ -659,6 +667,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         off[4 * c + 2] = bias - v.z;
         off[4 * c + 3] = bias - v.w;
       }
+      if (tq != nullptr) {
+        // query pruning: the 32-row quarters of the tile that do not keep this key
+        // block give it probability 0 (columns 32 h .. 32 h + 31 of this warpgroup)
+        const uint32_t bits = tq[t];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (((bits >> (2 * w + h)) & 1u) == 0u) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) off[32 * h + k] = -INFINITY;
+          }
+      }
       if (!wait_warp(br.s_full(0), t & 1)) {
         failed = true;
         break;
@@ -784,10 +803,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ------------------------------------------------------------------ preparation
 
-// fp16 copies of Q and K (8 elements per step), lse2 padded to whole blocks, D cleared
+// fp16 copies of Q and K (8 elements per step; n8q and n8k pieces), lse2 padded to
+// whole blocks (all +inf when lse is null: the pruned backward scatters the kept
+// rows' values afterwards), D cleared
 __global__ void __launch_bounds__(256)
-    bwd_prep_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
-                    uint4* __restrict__ q16, uint4* __restrict__ k16, int64_t n8,
+    bwd_prep_kernel(const uint4* __restrict__ q, uint4* __restrict__ q16, int64_t n8q,
+                    const uint4* __restrict__ k, uint4* __restrict__ k16, int64_t n8k,
                     const float* __restrict__ lse, float* __restrict__ lse2,
                     float* __restrict__ Dvec, int BH, int N, int Np,
                     unsigned int* __restrict__ err_word) {
@@ -799,16 +820,19 @@ __global__ void __launch_bounds__(256)
     bad |= ((h & 0x7c00u) == 0x7c00u) | ((h & 0x7c000000u) == 0x7c000000u);
     return h;
   };
-  for (int64_t j = i0; j < n8; j += stride) {
-    const uint4 a = q[j], b = k[j];
+  for (int64_t j = i0; j < n8q; j += stride) {
+    const uint4 a = q[j];
     q16[j] = make_uint4(cvt(a.x), cvt(a.y), cvt(a.z), cvt(a.w));
+  }
+  for (int64_t j = i0; j < n8k; j += stride) {
+    const uint4 b = k[j];
     k16[j] = make_uint4(cvt(b.x), cvt(b.y), cvt(b.z), cvt(b.w));
   }
   const int64_t nv = static_cast<int64_t>(BH) * Np;
   for (int64_t j = i0; j < nv; j += stride) {
     const int64_t h = j / Np;
     const int r = static_cast<int>(j - h * Np);
-    lse2[j] = r < N ? lse[h * N + r] * kLog2e : INFINITY;
+    lse2[j] = (lse != nullptr && r < N) ? lse[h * N + r] * kLog2e : INFINITY;
     Dvec[j] = 0.f;
   }
   if (__any_sync(0xffffffffu, bad != 0) && (threadIdx.x & 31) == 0) atomicOr(err_word, kErrRange);
@@ -834,9 +858,11 @@ __global__ void __launch_bounds__(256)
 
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace pieces (256-byte aligned, in this order): lse2, D [BH][nb*128] f32; Q16,
-// K16 [BH][N][d] f16; launch orders of query and key blocks [BH*nb] i32; with ASA_G
-// (G global tokens): Kg, Vg [BH][G][d] bf16, Kg16 [BH][G][d] f16, dKg, dVg [BH][G][d] f32.
+// Workspace pieces (256-byte aligned, in this order): lse2, D [BH][nbq*128] f32; Q16
+// [BH][Nq][d] f16, K16 [BH][N][d] f16; launch orders of query and key blocks
+// [BH*nbq], [BH*nbk] i32; with ASA_G (G global tokens): Kg, Vg [BH][G][d] bf16, Kg16
+// [BH][G][d] f16, dKg, dVg [BH][G][d] f32.  Without pruning Nq = N; with it Nq = Ns,
+// the compact query rows, and the pruned pieces follow (carve_pruned).
 struct BwdWs {
   float *lse2, *Dvec;
   void *q16, *k16;
@@ -846,8 +872,9 @@ struct BwdWs {
   size_t bytes;
 };
 
-BwdWs carve_bwd(void* base, int BH, int N, int d, int G) {
-  const size_t nb = (static_cast<size_t>(N) + kBlock - 1) / kBlock;
+BwdWs carve_bwd(void* base, int BH, int Nq, int N, int d, int G) {
+  const size_t nbq = (static_cast<size_t>(Nq) + kBlock - 1) / kBlock;
+  const size_t nbk = (static_cast<size_t>(N) + kBlock - 1) / kBlock;
   char* w = static_cast<char*>(base);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -856,12 +883,12 @@ BwdWs carve_bwd(void* base, int BH, int N, int d, int G) {
     return p;
   };
   BwdWs r{};
-  r.lse2 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nb * kBlock * 4));
-  r.Dvec = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nb * kBlock * 4));
-  r.q16 = take(static_cast<size_t>(BH) * N * d * 2);
+  r.lse2 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nbq * kBlock * 4));
+  r.Dvec = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * nbq * kBlock * 4));
+  r.q16 = take(static_cast<size_t>(BH) * Nq * d * 2);
   r.k16 = take(static_cast<size_t>(BH) * N * d * 2);
-  r.ord_r = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nb * 4));
-  r.ord_c = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nb * 4));
+  r.ord_r = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nbq * 4));
+  r.ord_c = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nbk * 4));
   if (G > 0) {
     const size_t gd = static_cast<size_t>(BH) * G * d;
     r.kg = take(gd * 2);
@@ -874,23 +901,28 @@ BwdWs carve_bwd(void* base, int BH, int N, int d, int G) {
   return r;
 }
 
-template <int D>
+// Query side: Nq rows in nbq blocks (CSR row_ptr/col_idx over them, quarter bits
+// `quarters` with query pruning); key side: N rows in nbk blocks (transposed CSR
+// col_ptr_t/row_idx_t, quarter bits `tquarters`).
+template <int D, bool kPruned>
 cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
-                           const int32_t* col_idx, const int32_t* col_ptr_t,
-                           const int32_t* row_idx_t, const BwdWs& ws, int BH, int N, int G,
-                           int gw, void* dq, void* dk, void* dv, unsigned int* err_word,
+                           const int32_t* col_idx, const uint8_t* quarters,
+                           const int32_t* col_ptr_t, const int32_t* row_idx_t,
+                           const uint8_t* tquarters, const BwdWs& ws, int BH, int N, int Nq,
+                           int G, int gw, void* dq, void* dk, void* dv, unsigned int* err_word,
                            cudaStream_t stream) {
   using L = BwdLayout<D>;
-  const int nb = (N + kBlock - 1) / kBlock;
-  const int Np = nb * kBlock;
+  const int nbq = (Nq + kBlock - 1) / kBlock;
+  const int nbk = (N + kBlock - 1) / kBlock;
+  const int Np = nbq * kBlock;
   const float c2 = kLog2e / sqrtf(static_cast<float>(D));
   const float scale = 1.f / sqrtf(static_cast<float>(D));
   const float gbias2 = gw > 0 ? log2f(static_cast<float>(gw)) : 0.f;
   const long long limit = 1ll << 31;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_row_kernel<D, true>,
+  if ((e = cudaFuncSetAttribute(bwd_row_kernel<D, true, kPruned>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
-      (e = cudaFuncSetAttribute(bwd_row_kernel<D, false>,
+      (e = cudaFuncSetAttribute(bwd_row_kernel<D, false, kPruned>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
       (e = cudaFuncSetAttribute(bwd_col_kernel<D, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem)) ||
@@ -899,8 +931,8 @@ cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
     return e;
   static int regs_checked = 0;
   if (regs_checked == 0) {
-    const void* fns[4] = {reinterpret_cast<const void*>(bwd_row_kernel<D, true>),
-                          reinterpret_cast<const void*>(bwd_row_kernel<D, false>),
+    const void* fns[4] = {reinterpret_cast<const void*>(bwd_row_kernel<D, true, kPruned>),
+                          reinterpret_cast<const void*>(bwd_row_kernel<D, false, kPruned>),
                           reinterpret_cast<const void*>(bwd_col_kernel<D, false>),
                           reinterpret_cast<const void*>(bwd_col_kernel<D, true>)};
     regs_checked = 1;
@@ -911,29 +943,91 @@ cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
     }
   }
   if (regs_checked < 0) return cudaErrorInvalidConfiguration;
-  const int grid = BH * nb;
+  const int grid_q = BH * nbq, grid_k = BH * nbk;
   // maps: Q16, dO, K16, V, Kg16, Vg (the last two stand in for K16, V without ASA_G)
-  bwd_row_kernel<D, true><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, ws.ord_r, N, nb,
-      Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, err_word, limit);
+  bwd_row_kernel<D, true, kPruned><<<grid_q, kBwdThreads, L::kSmem, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, quarters, ws.ord_r,
+      N, Nq, nbq, Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, err_word, limit);
   if ((e = cudaGetLastError())) return e;
   if (G > 0) {
     const int gtiles = BH * ((G + kBlock - 1) / kBlock);
     bwd_col_kernel<D, true><<<gtiles, kBwdThreads, L::kSmem, stream>>>(
-        maps[4], maps[5], maps[0], maps[1], col_ptr_t, row_idx_t, ws.ord_c, N, nb, Np, G, gw,
-        gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, nullptr, ws.dkg, ws.dvg, err_word, limit);
+        maps[4], maps[5], maps[0], maps[1], col_ptr_t, row_idx_t, nullptr, ws.ord_c, N, nbk, nbq,
+        Np, G, gw, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, nullptr, ws.dkg, ws.dvg,
+        err_word, limit);
     if ((e = cudaGetLastError())) return e;
   }
-  bwd_col_kernel<D, false><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[2], maps[3], maps[0], maps[1], col_ptr_t, row_idx_t, ws.ord_c, N, nb, Np, G, gw,
-      gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dk),
+  bwd_col_kernel<D, false><<<grid_k, kBwdThreads, L::kSmem, stream>>>(
+      maps[2], maps[3], maps[0], maps[1], col_ptr_t, row_idx_t, tquarters, ws.ord_c, N, nbk, nbq,
+      Np, G, gw, gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv), ws.dkg, ws.dvg, err_word, limit);
   if ((e = cudaGetLastError())) return e;
-  bwd_row_kernel<D, false><<<grid, kBwdThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, ws.ord_r, N, nb,
-      Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dq), err_word,
-      limit);
+  bwd_row_kernel<D, false, kPruned><<<grid_q, kBwdThreads, L::kSmem, stream>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, quarters, ws.ord_r,
+      N, Nq, nbq, Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, static_cast<__nv_bfloat16*>(dq),
+      err_word, limit);
   return cudaGetLastError();
+}
+
+// Tensor maps of the backward: Q16 (Nq rows), dO (Nq rows), K16, V (N rows) and the
+// ASA_G global tokens (or K16, V again).
+bool make_bwd_maps(CUtensorMap* maps, const BwdWs& ws, const void* dout, const void* vp, int BH,
+                   int Nq, int N, int G, int d) {
+  if (!make_map_rows_f16(&maps[0], ws.q16, BH, Nq, d) || !make_map_rows(&maps[1], dout, BH, Nq, d) ||
+      !make_map_rows_f16(&maps[2], ws.k16, BH, N, d) || !make_map_rows(&maps[3], vp, BH, N, d))
+    return false;
+  if (G > 0)
+    return make_map_rows_f16(&maps[4], ws.kg16, BH, G, d) && make_map_rows(&maps[5], ws.vg, BH, G, d);
+  maps[4] = maps[2];
+  maps[5] = maps[3];
+  return true;
+}
+
+// the forward's global tokens, recomputed: mean-pooled K and V, Kg also in fp16
+cudaError_t global_tokens(const void* kp, const void* vp, const BwdWs& ws, int BH, int N, int d,
+                          int gw, int G, unsigned int* err_word, int num_sms, cudaStream_t stream) {
+  cudaError_t e = launch_global_pool(kp, ws.kg, BH, N, d, gw, num_sms, stream);
+  if (e == cudaSuccess) e = launch_global_pool(vp, ws.vg, BH, N, d, gw, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  f16_copy_kernel<<<num_sms * 8, 256, 0, stream>>>(static_cast<const uint4*>(ws.kg),
+                                                   static_cast<uint4*>(ws.kg16),
+                                                   static_cast<int64_t>(BH) * G * d / 8, err_word);
+  return cudaGetLastError();
+}
+
+// The pruned backward's own pieces, after carve_bwd's: dO' and dQ in the compact
+// layout [BH][Ns][d] bf16; the dense quarter matrix [BH][ntile][nbk] u8; the
+// transposed tile CSR (counts [BH*nbk], col_ptr [BH*nbk + 1], tile index and quarter
+// bits with room for every (tile, key block) pair).
+struct PrunedWs {
+  void *dout_s, *dq_s;
+  uint8_t* qmat;
+  int32_t *counts, *tcol_ptr, *trow_idx;
+  uint8_t* tquarters;
+  size_t bytes;
+};
+
+PrunedWs carve_pruned(void* base, size_t start, int BH, int N, int Ns, int d) {
+  const size_t ntile = static_cast<size_t>(Ns) / kBlock;
+  const size_t nbk = (static_cast<size_t>(N) + kBlock - 1) / kBlock;
+  char* w = static_cast<char*>(base);
+  size_t off = start;
+  auto take = [&](size_t bytes) {
+    char* p = w == nullptr ? nullptr : w + off;
+    off += a256(bytes);
+    return p;
+  };
+  PrunedWs r{};
+  const size_t pairs = static_cast<size_t>(BH) * ntile * nbk;
+  r.dout_s = take(static_cast<size_t>(BH) * Ns * d * 2);
+  r.dq_s = take(static_cast<size_t>(BH) * Ns * d * 2);
+  r.qmat = reinterpret_cast<uint8_t*>(take(pairs));
+  r.counts = reinterpret_cast<int32_t*>(take(static_cast<size_t>(BH) * nbk * 4));
+  r.tcol_ptr = reinterpret_cast<int32_t*>(take((static_cast<size_t>(BH) * nbk + 1) * 4));
+  r.trow_idx = reinterpret_cast<int32_t*>(take(pairs * 4));
+  r.tquarters = reinterpret_cast<uint8_t*>(take(pairs));
+  r.bytes = off;
+  return r;
 }
 
 }  // namespace
@@ -941,7 +1035,14 @@ cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
 size_t bwd_tc_workspace_bytes(int BH, int N, int d, int global_window) {
   if (BH < 1 || N < 1 || global_window < 0) return 0;
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
-  return carve_bwd(nullptr, BH, N, d, G).bytes;
+  return carve_bwd(nullptr, BH, N, N, d, G).bytes;
+}
+
+size_t bwd_tc_pruned_workspace_bytes(int BH, int N, int Ns, int d, int global_window) {
+  if (BH < 1 || N < 1 || Ns < kBlock || Ns % kBlock != 0 || global_window < 0) return 0;
+  const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
+  const size_t base = carve_bwd(nullptr, BH, Ns, N, d, G).bytes;
+  return carve_pruned(nullptr, base, BH, N, Ns, d).bytes;
 }
 
 cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const void* dout,
@@ -953,47 +1054,72 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
   const int Np = nb * kBlock;
   const int gw = global_window;
   const int G = gw > 0 ? (N + gw - 1) / gw : 0;
-  const BwdWs ws = carve_bwd(workspace, BH, N, d, G);
-
+  const BwdWs ws = carve_bwd(workspace, BH, N, N, d, G);
   CUtensorMap maps[6];
-  if (!make_map_rows_f16(&maps[0], ws.q16, BH, N, d) ||
-      !make_map_rows(&maps[1], dout, BH, N, d) ||
-      !make_map_rows_f16(&maps[2], ws.k16, BH, N, d) || !make_map_rows(&maps[3], vp, BH, N, d))
-    return cudaErrorInvalidValue;
-  if (G > 0) {
-    if (!make_map_rows_f16(&maps[4], ws.kg16, BH, G, d) ||
-        !make_map_rows(&maps[5], ws.vg, BH, G, d))
-      return cudaErrorInvalidValue;
-  } else {
-    maps[4] = maps[2];
-    maps[5] = maps[3];
-  }
-
-  const int blocks = num_sms * 8;
-  bwd_prep_kernel<<<blocks, 256, 0, stream>>>(
-      static_cast<const uint4*>(qp), static_cast<const uint4*>(kp), static_cast<uint4*>(ws.q16),
-      static_cast<uint4*>(ws.k16), static_cast<int64_t>(BH) * N * d / 8, lse, ws.lse2, ws.Dvec,
-      BH, N, Np, err_word);
+  if (!make_bwd_maps(maps, ws, dout, vp, BH, N, N, G, d)) return cudaErrorInvalidValue;
+  const int64_t n8 = static_cast<int64_t>(BH) * N * d / 8;
+  bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(
+      static_cast<const uint4*>(qp), static_cast<uint4*>(ws.q16), n8,
+      static_cast<const uint4*>(kp), static_cast<uint4*>(ws.k16), n8, lse, ws.lse2, ws.Dvec, BH,
+      N, Np, err_word);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess && G > 0) {
-    // the forward's global tokens, recomputed: mean-pooled K and V, Kg also in fp16
-    e = launch_global_pool(kp, ws.kg, BH, N, d, gw, num_sms, stream);
-    if (e == cudaSuccess) e = launch_global_pool(vp, ws.vg, BH, N, d, gw, num_sms, stream);
-    if (e == cudaSuccess) {
-      f16_copy_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(ws.kg),
-                                                  static_cast<uint4*>(ws.kg16),
-                                                  static_cast<int64_t>(BH) * G * d / 8, err_word);
-      e = cudaGetLastError();
-    }
-  }
+  if (e == cudaSuccess && G > 0) e = global_tokens(kp, vp, ws, BH, N, d, gw, G, err_word, num_sms, stream);
   if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, nb, ws.ord_r, stream);
   if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, nb, ws.ord_c, stream);
   if (e != cudaSuccess) return e;
   if (d == 128)
-    return launch_kernels<128>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ws, BH, N, G, gw,
-                               dq, dk, dv, err_word, stream);
-  return launch_kernels<64>(maps, row_ptr, col_idx, col_ptr_t, row_idx_t, ws, BH, N, G, gw, dq,
-                            dk, dv, err_word, stream);
+    return launch_kernels<128, false>(maps, row_ptr, col_idx, nullptr, col_ptr_t, row_idx_t,
+                                      nullptr, ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream);
+  return launch_kernels<64, false>(maps, row_ptr, col_idx, nullptr, col_ptr_t, row_idx_t, nullptr,
+                                   ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream);
+}
+
+// Backward with query pruning on the packed tiles of the pruned forward: the query
+// side runs over the compact rows (Ns per head: ntile tiles), each (tile, key block)
+// entry restricted to the lane quarters whose block keeps it; the key side walks the
+// transposed tile CSR.  Work is proportional to the packed forward's.
+cudaError_t launch_bwd_tc_pruned(const void* q_s, const void* kp, const void* vp, const void* dout,
+                                 const float* lse, const int32_t* src_pos, const int32_t* src_row,
+                                 const int32_t* tile_ptr, const int32_t* tile_col,
+                                 const uint8_t* tile_quarters, int BH, int N, int Ns, int d,
+                                 int global_window, void* workspace, void* dq, void* dk, void* dv,
+                                 unsigned int* err_word, int num_sms, cudaStream_t stream) {
+  const int ntile = Ns / kBlock;
+  const int nbk = (N + kBlock - 1) / kBlock;
+  const int gw = global_window;
+  const int G = gw > 0 ? (N + gw - 1) / gw : 0;
+  const BwdWs ws = carve_bwd(workspace, BH, Ns, N, d, G);
+  const PrunedWs pw = carve_pruned(workspace, ws.bytes, BH, N, Ns, d);
+  CUtensorMap maps[6];
+  if (!make_bwd_maps(maps, ws, pw.dout_s, vp, BH, Ns, N, G, d)) return cudaErrorInvalidValue;
+  // compact dO' (unused rows zero) and lse2 (unused rows +inf: probability 0)
+  cudaError_t e = cudaMemsetAsync(pw.dout_s, 0, static_cast<size_t>(BH) * Ns * d * 2, stream);
+  if (e != cudaSuccess) return e;
+  bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(
+      static_cast<const uint4*>(q_s), static_cast<uint4*>(ws.q16),
+      static_cast<int64_t>(BH) * Ns * d / 8, static_cast<const uint4*>(kp),
+      static_cast<uint4*>(ws.k16), static_cast<int64_t>(BH) * N * d / 8, nullptr, ws.lse2, ws.Dvec,
+      BH, Ns, Ns, err_word);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_dout_compact(dout, lse, src_pos, src_row, BH, N, Ns, d, pw.dout_s, ws.lse2, err_word,
+                          num_sms, stream);
+  if (e == cudaSuccess && G > 0) e = global_tokens(kp, vp, ws, BH, N, d, gw, G, err_word, num_sms, stream);
+  if (e == cudaSuccess)
+    e = launch_tile_transpose(tile_ptr, tile_col, tile_quarters, BH, ntile, nbk, pw.qmat, pw.counts,
+                              pw.tcol_ptr, pw.trow_idx, pw.tquarters, err_word, num_sms, stream);
+  if (e == cudaSuccess) e = launch_lpt_order(tile_ptr, BH, ntile, nbk, ws.ord_r, stream);
+  if (e == cudaSuccess) e = launch_lpt_order(pw.tcol_ptr, BH, nbk, ntile, ws.ord_c, stream);
+  if (e != cudaSuccess) return e;
+  if (d == 128)
+    e = launch_kernels<128, true>(maps, tile_ptr, tile_col, tile_quarters, pw.tcol_ptr,
+                                  pw.trow_idx, pw.tquarters, ws, BH, N, Ns, G, gw, pw.dq_s, dk, dv,
+                                  err_word, stream);
+  else
+    e = launch_kernels<64, true>(maps, tile_ptr, tile_col, tile_quarters, pw.tcol_ptr, pw.trow_idx,
+                                 pw.tquarters, ws, BH, N, Ns, G, gw, pw.dq_s, dk, dv, err_word,
+                                 stream);
+  if (e != cudaSuccess) return e;
+  return launch_dq_scatter(pw.dq_s, src_pos, src_row, BH, N, Ns, d, dq, err_word, num_sms, stream);
 }
 
 }  // namespace asa

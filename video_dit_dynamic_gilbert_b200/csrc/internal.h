@@ -87,9 +87,21 @@ cudaError_t launch_prune_mask(const int32_t* row_ptr, const int32_t* col_idx, in
 cudaError_t launch_fill_out(const void* o_s, const float* lse_s, const int32_t* src_row, int BH,
                             int N, int Ns, int d, void* o, float* lse, unsigned int* err_word,
                             int num_sms, cudaStream_t stream);
-cudaError_t launch_dout_fill(const void* dout, const float* lse, const int32_t* src_pos, int BH,
-                             int N, int d, void* dout2, float* lse2, unsigned int* err_word,
-                             int num_sms, cudaStream_t stream);
+// Pruned backward inputs in the compact layout (dO' sums and lse2 of the kept rows).
+cudaError_t launch_dout_compact(const void* dout, const float* lse, const int32_t* src_pos,
+                                const int32_t* src_row, int BH, int N, int Ns, int d,
+                                void* dout_s, float* lse2_s, unsigned int* err_word, int num_sms,
+                                cudaStream_t stream);
+cudaError_t launch_dq_scatter(const void* dq_s, const int32_t* src_pos, const int32_t* src_row,
+                              int BH, int N, int Ns, int d, void* dq, unsigned int* err_word,
+                              int num_sms, cudaStream_t stream);
+// Transposed tile CSR (per key block, the tiles holding it) through a dense
+// [BH][ntile][nbk] quarter matrix qmat; counts: [BH * nbk] scratch.
+cudaError_t launch_tile_transpose(const int32_t* tile_ptr, const int32_t* tile_col,
+                                  const uint8_t* tile_quarters, int BH, int ntile, int nbk,
+                                  uint8_t* qmat, int32_t* counts, int32_t* tcol_ptr,
+                                  int32_t* trow_idx, uint8_t* tquarters, unsigned int* err_word,
+                                  int num_sms, cudaStream_t stream);
 // Forward over a packed tile CSR: q_s has Ns rows per head; quarters[e] says which
 // 32-row lane quarters of the tile see entry e; o_s, lse_s: [BH][Ns].
 cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp,
@@ -98,6 +110,15 @@ cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp
                                  int32_t* order, int BH, int N, int Ns, int d, int global_window,
                                  void* o_s, float* lse_s, unsigned int* err_word,
                                  cudaStream_t stream);
+
+// Backward with query pruning on packed tiles (workspace: bwd_tc_pruned_workspace_bytes).
+size_t bwd_tc_pruned_workspace_bytes(int BH, int N, int Ns, int d, int global_window);
+cudaError_t launch_bwd_tc_pruned(const void* q_s, const void* kp, const void* vp, const void* dout,
+                                 const float* lse, const int32_t* src_pos, const int32_t* src_row,
+                                 const int32_t* tile_ptr, const int32_t* tile_col,
+                                 const uint8_t* tile_quarters, int BH, int N, int Ns, int d,
+                                 int global_window, void* workspace, void* dq, void* dk, void* dv,
+                                 unsigned int* err_word, int num_sms, cudaStream_t stream);
 
 // Failure-detection test hook: one bounded wait on a barrier nothing arrives at.
 cudaError_t launch_wait_timeout(unsigned int* err_word, long long limit, cudaStream_t stream);

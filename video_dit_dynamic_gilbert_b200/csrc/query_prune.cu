@@ -289,15 +289,17 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Backward inputs under pruning: dO'[i] = sum of dO[j] over the tokens j of i's block
-// with src_pos[j] = i when token i is kept (src_pos[i] = i), else 0; lse'[i] = lse[i]
-// for kept rows, +inf for pruned ones (their probabilities vanish).  One warp per row.
+// Backward inputs in the compact layout: for a kept token i (src_pos[i] = i) with
+// compact row r = src_row[i], dO'_s[r] = the sum of dO[j] over the tokens j of i's
+// block with src_pos[j] = i (its own gradient and those of the pruned tokens it
+// fills), stored in bf16, and lse2_s[r] = lse[i] log2(e).  One warp per token; a
+// pruned token only checks that it points at a kept token of its own block.
 template <int D>
 __global__ void __launch_bounds__(256)
-    dout_fill_kernel(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
-                     const int32_t* __restrict__ src_pos, int64_t rows, int N,
-                     __nv_bfloat16* __restrict__ dout2, float* __restrict__ lse2,
-                     unsigned int* __restrict__ err_word) {
+    dout_compact_kernel(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                        const int32_t* __restrict__ src_pos, const int32_t* __restrict__ src_row,
+                        int64_t rows, int N, int Ns, __nv_bfloat16* __restrict__ dout_s,
+                        float* __restrict__ lse2_s, unsigned int* __restrict__ err_word) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -309,34 +311,117 @@ __global__ void __launch_bounds__(256)
     const int L = min(kBlock, N - s0);
     const int32_t* sp = src_pos + bh * N;
     const int p = sp[i];
-    bool bad = p < s0 || p >= s0 + L || sp[p] != p;
+    if (p != i) {
+      const bool bad = p < s0 || p >= s0 + L || sp[p] != p;
+      if (bad && lane == 0) atomicOr(err_word, kErrBadIndex);
+      continue;
+    }
+    const int r = src_row[row];
+    if (r < 0 || r >= Ns) {
+      if (lane == 0) atomicOr(err_word, kErrBadIndex);
+      continue;
+    }
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    if (!bad && p == i) {
-      for (int j0 = 0; j0 < L; j0 += 32) {
-        const int j = j0 + lane;
-        unsigned m = __ballot_sync(0xffffffffu, j < L && sp[s0 + j] == i);
-        while (m != 0u) {
-          const int b = __ffs(m) - 1;
-          m &= m - 1u;
-          float x[E];
-          load_bf16<E>(dout + (bh * N + s0 + j0 + b) * D + lane * E, x);
+    for (int j0 = 0; j0 < L; j0 += 32) {
+      const int j = j0 + lane;
+      unsigned m = __ballot_sync(0xffffffffu, j < L && sp[s0 + j] == i);
+      while (m != 0u) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1u;
+        float x[E];
+        load_bf16<E>(dout + (bh * N + s0 + j0 + b) * D + lane * E, x);
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] += x[e];
-        }
+        for (int e = 0; e < E; ++e) acc[e] += x[e];
       }
     }
-    __nv_bfloat16* dst = dout2 + row * D + lane * E;
+    __nv_bfloat16* dst = dout_s + (bh * Ns + r) * D + lane * E;
     if constexpr (E == 4) {
       *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
     } else {
       *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0], acc[1]);
     }
-    if (lane == 0) {
-      lse2[row] = (!bad && p == i) ? lse[row] : INFINITY;
-      if (bad) atomicOr(err_word, kErrBadIndex);
+    if (lane == 0) lse2_s[bh * Ns + r] = lse[row] * kLog2e;
+  }
+}
+
+// dQ[i] = dQ_s[src_row[i]] for a kept token, 0 for a pruned one (its output is a copy
+// of its centre's, so its query gets no gradient).  D/8 threads per row.
+template <int D>
+__global__ void __launch_bounds__(256)
+    dq_scatter_kernel(const __nv_bfloat16* __restrict__ dq_s, const int32_t* __restrict__ src_pos,
+                      const int32_t* __restrict__ src_row, int64_t rows, int N, int Ns,
+                      __nv_bfloat16* __restrict__ dq, unsigned int* __restrict__ err_word) {
+  constexpr int kVec = D / 8;
+  const int64_t total = rows * kVec;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = g / kVec;
+    const int v = static_cast<int>(g - row * kVec);
+    const int64_t bh = row / N;
+    const int i = static_cast<int>(row - bh * N);
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (src_pos[row] == i) {
+      const int r = src_row[row];
+      if (r >= 0 && r < Ns)
+        x = reinterpret_cast<const uint4*>(dq_s + (bh * Ns + r) * D)[v];
+      else if (v == 0)
+        atomicOr(err_word, kErrBadIndex);
     }
+    reinterpret_cast<uint4*>(dq + row * D)[v] = x;
+  }
+}
+
+// Dense quarter matrix [BH][ntile][nbk] (zeroed by the caller) from the tile CSR:
+// one warp per tile row.
+__global__ void __launch_bounds__(256)
+    tile_dense_kernel(const int32_t* __restrict__ tile_ptr, const int32_t* __restrict__ tile_col,
+                      const uint8_t* __restrict__ tile_quarters, int rows, int nbk,
+                      uint8_t* __restrict__ qmat, unsigned int* __restrict__ err_word) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    bool bad = false;
+    for (int e = tile_ptr[r] + lane; e < tile_ptr[r + 1]; e += 32) {
+      const int J = tile_col[e];
+      if (J < 0 || J >= nbk) {
+        bad = true;
+        continue;
+      }
+      qmat[static_cast<int64_t>(r) * nbk + J] = tile_quarters[e];
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err_word, kErrBadIndex);
+  }
+}
+
+// Transposed tile CSR from the dense matrix: for each (bh, key block J) the tiles t
+// holding J, t ascending, with their quarter bits.  One warp per (bh, J), lanes over t.
+template <bool kFill>
+__global__ void __launch_bounds__(256)
+    tile_transpose_kernel(const uint8_t* __restrict__ qmat, int BH, int ntile, int nbk,
+                          int32_t* __restrict__ counts, const int32_t* __restrict__ tcol_ptr,
+                          int32_t* __restrict__ trow_idx, uint8_t* __restrict__ tquarters) {
+  const int lane = threadIdx.x & 31;
+  const int64_t cols = static_cast<int64_t>(BH) * nbk;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       c < cols; c += warps) {
+    const int64_t bh = c / nbk;
+    const int J = static_cast<int>(c - bh * nbk);
+    int pos = kFill ? tcol_ptr[c] : 0;
+    for (int t0 = 0; t0 < ntile; t0 += 32) {
+      const int t = t0 + lane;
+      const uint8_t q = t < ntile ? qmat[(bh * ntile + t) * nbk + J] : 0;
+      const unsigned m = __ballot_sync(0xffffffffu, q != 0);
+      if (kFill && q != 0) {
+        const int p = pos + __popc(m & ((1u << lane) - 1u));
+        trow_idx[p] = t;
+        tquarters[p] = q;
+      }
+      pos += __popc(m);
+    }
+    if (!kFill && lane == 0) counts[c] = pos;
   }
 }
 
@@ -396,17 +481,57 @@ cudaError_t launch_fill_out(const void* o_s, const float* lse_s, const int32_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_dout_fill(const void* dout, const float* lse, const int32_t* src_pos, int BH,
-                             int N, int d, void* dout2, float* lse2, unsigned int* err_word,
-                             int num_sms, cudaStream_t stream) {
+cudaError_t launch_dout_compact(const void* dout, const float* lse, const int32_t* src_pos,
+                                const int32_t* src_row, int BH, int N, int Ns, int d,
+                                void* dout_s, float* lse2_s, unsigned int* err_word, int num_sms,
+                                cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(BH) * N;
   const unsigned grid = grid_of(rows, 8, num_sms, 8);
   const auto* src = static_cast<const __nv_bfloat16*>(dout);
-  auto* dst = static_cast<__nv_bfloat16*>(dout2);
+  auto* dst = static_cast<__nv_bfloat16*>(dout_s);
   if (d == 128)
-    dout_fill_kernel<128><<<grid, 256, 0, stream>>>(src, lse, src_pos, rows, N, dst, lse2, err_word);
+    dout_compact_kernel<128><<<grid, 256, 0, stream>>>(src, lse, src_pos, src_row, rows, N, Ns, dst,
+                                                       lse2_s, err_word);
   else
-    dout_fill_kernel<64><<<grid, 256, 0, stream>>>(src, lse, src_pos, rows, N, dst, lse2, err_word);
+    dout_compact_kernel<64><<<grid, 256, 0, stream>>>(src, lse, src_pos, src_row, rows, N, Ns, dst,
+                                                      lse2_s, err_word);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_scatter(const void* dq_s, const int32_t* src_pos, const int32_t* src_row,
+                              int BH, int N, int Ns, int d, void* dq, unsigned int* err_word,
+                              int num_sms, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(BH) * N;
+  const unsigned grid = grid_of(rows * (d / 8), 256, num_sms, 8);
+  const auto* src = static_cast<const __nv_bfloat16*>(dq_s);
+  auto* dst = static_cast<__nv_bfloat16*>(dq);
+  if (d == 128)
+    dq_scatter_kernel<128><<<grid, 256, 0, stream>>>(src, src_pos, src_row, rows, N, Ns, dst, err_word);
+  else
+    dq_scatter_kernel<64><<<grid, 256, 0, stream>>>(src, src_pos, src_row, rows, N, Ns, dst, err_word);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_transpose(const int32_t* tile_ptr, const int32_t* tile_col,
+                                  const uint8_t* tile_quarters, int BH, int ntile, int nbk,
+                                  uint8_t* qmat, int32_t* counts, int32_t* tcol_ptr,
+                                  int32_t* trow_idx, uint8_t* tquarters, unsigned int* err_word,
+                                  int num_sms, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(BH) * ntile;
+  cudaError_t e = cudaMemsetAsync(qmat, 0, static_cast<size_t>(rows) * nbk, stream);
+  if (e != cudaSuccess) return e;
+  tile_dense_kernel<<<grid_of(rows, 8, num_sms, 8), 256, 0, stream>>>(
+      tile_ptr, tile_col, tile_quarters, static_cast<int>(rows), nbk, qmat, err_word);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t cols = static_cast<int64_t>(BH) * nbk;
+  const unsigned grid = grid_of(cols, 8, num_sms, 8);
+  tile_transpose_kernel<false><<<grid, 256, 0, stream>>>(qmat, BH, ntile, nbk, counts, nullptr,
+                                                         nullptr, nullptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_scan(counts, static_cast<int>(cols), tcol_ptr, nullptr, stream)) != cudaSuccess)
+    return e;
+  tile_transpose_kernel<true><<<grid, 256, 0, stream>>>(qmat, BH, ntile, nbk, nullptr, tcol_ptr,
+                                                        trow_idx, tquarters);
   return cudaGetLastError();
 }
 
