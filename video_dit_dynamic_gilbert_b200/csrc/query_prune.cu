@@ -66,9 +66,21 @@ __global__ void __launch_bounds__(kPruneThreads)
   const __nv_bfloat16* qb = qp + (static_cast<int64_t>(bh) * N + s0) * D;
   constexpr int kVec = D / 8;  // 16-byte pieces per row
   {
+    // every load in flight before the first store (8 or 4 pieces per thread)
+    constexpr int kPer = kBlock * kVec / kPruneThreads;
     const uint4* src = reinterpret_cast<const uint4*>(qb);
     uint4* dst = reinterpret_cast<uint4*>(s_q);
-    for (int i = tid; i < L * kVec; i += kPruneThreads) dst[i] = src[i];
+    uint4 v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kPruneThreads;
+      if (i < L * kVec) v[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kPruneThreads;
+      if (i < L * kVec) dst[i] = v[u];
+    }
   }
   __syncthreads();
   auto centre = [&](int t) {
