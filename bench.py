@@ -370,6 +370,35 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
         tb = r["attn_bwd"]["median_ms"] * 1e-3
         r["attn_bwd"]["effective_TFLOP_s"] = 2.5 * flops / tb / 1e12
         r["attn_bwd"]["executed_TFLOP_s"] = 4.5 * flops / tb / 1e12
+    # BSA query pruning with token filling on the same mask: r = 0.5, windows of 8
+    pr = asa.asa_prune_queries(qp, 0.5, 8)
+    pmws = asa._workspace(asa.lib().asa_prune_mask_workspace_size(B, H, N, pr.pack), dev)
+    ptm = asa.asa_prune_mask(mask, pr.pack, workspace=pmws)
+    pfws = asa.fwd_pruned_workspace(B, H, N, d, pr.pack, gw, dev)
+    plse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    qpr = {"r": 0.5, "window": 8, "pack": pr.pack}
+    qpr["prune"] = timer(lambda: asa.asa_prune_queries(qp, 0.5, 8, out=pr))
+    qpr["prune"]["GB_s"] = (tensor_bytes + B * H * pr.Ns * d * 2 + 2 * B * H * N * 4) / (
+        qpr["prune"]["median_ms"] * 1e-3) / 1e9
+    qpr["prune_mask"] = timer(lambda: asa.asa_prune_mask(mask, pr.pack, workspace=pmws, out=ptm))
+    qpr["attn_fwd"] = timer(lambda: asa.asa_sparse_attn_fwd_pruned(pr, kp, vp, ptm, global_window=gw,
+                                                                   workspace=pfws, out=op, lse=plse))
+    torch.cuda.synchronize()
+    pflops, nkept = _pruned_flops(mask.row_ptr.cpu().numpy(), mask.col_idx.cpu().numpy(),
+                                  pr.src_pos.cpu().numpy(), B, H, N, d)
+    if gw > 0:
+        pflops += 4 * d * nkept * (-(-N // gw))
+    qpr.update({"kept_queries": nkept, "tile_entries": int(ptm.nnz.item()),
+                "block_entries": nnz, "effective_flops": pflops,
+                "fwd_speedup": r["attn_fwd"]["median_ms"] / qpr["attn_fwd"]["median_ms"]})
+    qpr["attn_fwd"]["TFLOP_s"] = pflops / (qpr["attn_fwd"]["median_ms"] * 1e-3) / 1e12
+    if want_bwd:
+        pbws = asa.bwd_pruned_workspace(B, H, N, d, pr.pack, dev, gw)
+        qpr["attn_bwd"] = timer(lambda: asa.asa_sparse_attn_bwd_pruned(
+            pr, kp, vp, dop, plse, ptm, global_window=gw, workspace=pbws, outs=grads), reps=8, warm=3)
+        qpr["attn_bwd"]["effective_TFLOP_s"] = 2.5 * pflops / (qpr["attn_bwd"]["median_ms"] * 1e-3) / 1e12
+        qpr["bwd_speedup"] = r["attn_bwd"]["median_ms"] / qpr["attn_bwd"]["median_ms"]
+    r["query_prune"] = qpr
     asa.asa_check_device_status()
     return r, (qp, kp, vp)
 
@@ -443,6 +472,11 @@ def run_report(path):
         if "attn_bwd" in r:
             line += (f" bwd {r['attn_bwd']['median_ms']:.2f} ms "
                      f"{r['attn_bwd']['effective_TFLOP_s']:.0f} TF/s eff")
+        qpr = r["query_prune"]
+        line += (f" | pruned r=0.5: fwd {qpr['attn_fwd']['median_ms']:.3f} ms "
+                 f"(x{qpr['fwd_speedup']:.2f})")
+        if "attn_bwd" in qpr:
+            line += f" bwd {qpr['attn_bwd']['median_ms']:.2f} ms (x{qpr['bwd_speedup']:.2f})"
         print(line)
     return rep
 
