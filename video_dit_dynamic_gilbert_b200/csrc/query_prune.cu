@@ -46,15 +46,18 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 constexpr int kPruneThreads = 256;
 constexpr int kPruneWarps = kPruneThreads / 32;
 
-// One CTA per (b, h, block I).  The block's queries are staged in shared memory with
-// independent 16-byte loads; each warp then takes tokens t = warp, warp + 8, ... and
-// reads rows t and centre(t) from shared memory (one contiguous row per warp access).
+// One CTA per (b, h, block I), two threads per token.  The block's queries are staged
+// in shared memory (every load in flight before the stores); 16-byte piece c of row t
+// is stored at piece c ^ (t mod kVec), so that the threads of a warp, each reading its
+// own row, spread over all banks.  Thread pair (2t, 2t + 1) computes token t's dot
+// products over one half of d each and ranks it against one half of the block.
 template <int D>
 __global__ void __launch_bounds__(kPruneThreads)
     prune_kernel(const __nv_bfloat16* __restrict__ qp, int N, int nb, float r, int w, int pack,
                  __nv_bfloat16* __restrict__ q_s, int Ns, int32_t* __restrict__ src_pos,
                  int32_t* __restrict__ src_row) {
-  __shared__ __align__(16) __nv_bfloat16 s_q[kBlock * D];
+  constexpr int kVec = D / 8;  // 16-byte pieces per row
+  __shared__ uint4 s_q[kBlock * kVec];
   __shared__ float s_dis[kBlock];
   __shared__ int s_slot[kBlock];
   __shared__ int s_tok[kBlock];
@@ -64,12 +67,10 @@ __global__ void __launch_bounds__(kPruneThreads)
   const int s0 = I * kBlock;
   const int L = min(kBlock, N - s0);
   const __nv_bfloat16* qb = qp + (static_cast<int64_t>(bh) * N + s0) * D;
-  constexpr int kVec = D / 8;  // 16-byte pieces per row
+  auto piece = [](int row, int c) { return row * kVec + (c ^ (row & (kVec - 1))); };
   {
-    // every load in flight before the first store (8 or 4 pieces per thread)
     constexpr int kPer = kBlock * kVec / kPruneThreads;
     const uint4* src = reinterpret_cast<const uint4*>(qb);
-    uint4* dst = reinterpret_cast<uint4*>(s_q);
     uint4 v[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kPruneThreads)
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = tid + u * kPruneThreads;
-      if (i < L * kVec) dst[i] = v[u];
+      if (i < L * kVec) s_q[piece(i / kVec, i % kVec)] = v[u];
     }
   }
   __syncthreads();
@@ -88,53 +89,59 @@ __global__ void __launch_bounds__(kPruneThreads)
     return ws + min(w, L - ws) / 2;
   };
 
-  // 1 - cos(q_centre, q_t) in fp32, D/32 elements per lane; centres are kept
-  // unconditionally: -inf keeps them out of the ranking
-  constexpr int E = D / 32;
-  for (int t = warp; t < L; t += kPruneWarps) {
-    const int c = centre(t);
-    if (c == t) {
-      if (lane == 0) s_dis[t] = -INFINITY;
-      continue;
-    }
-    float a[E], b[E];
-    load_bf16<E>(s_q + t * D + lane * E, a);
-    load_bf16<E>(s_q + c * D + lane * E, b);
+  // 1 - cos(q_centre, q_t) in fp32; centres are kept unconditionally: -inf keeps them
+  // out of the ranking
+  const int t = tid >> 1, half = tid & 1;
+  {
     float dot = 0.f, na = 0.f, nc = 0.f;
+    const int c = t < L ? centre(t) : 0;
+    if (t < L && c != t) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      dot = fmaf(a[e], b[e], dot);
-      na = fmaf(a[e], a[e], na);
-      nc = fmaf(b[e], b[e], nc);
+      for (int j = 0; j < kVec / 2; ++j) {
+        const int pc = half * (kVec / 2) + j;
+        const uint4 a4 = s_q[piece(t, pc)], b4 = s_q[piece(c, pc)];
+        const uint32_t av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = __uint_as_float(av[e] << 16), a1 = __uint_as_float(av[e] & 0xffff0000u);
+          const float b0 = __uint_as_float(bv[e] << 16), b1 = __uint_as_float(bv[e] & 0xffff0000u);
+          dot = fmaf(a0, b0, fmaf(a1, b1, dot));
+          na = fmaf(a0, a0, fmaf(a1, a1, na));
+          nc = fmaf(b0, b0, fmaf(b1, b1, nc));
+        }
+      }
     }
-    dot = warp_sum_f(dot);
-    na = warp_sum_f(na);
-    nc = warp_sum_f(nc);
-    const float den = fmaxf(sqrtf(na), kCosEps) * fmaxf(sqrtf(nc), kCosEps);
-    if (lane == 0) s_dis[t] = 1.f - dot / den;
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    na += __shfl_xor_sync(0xffffffffu, na, 1);
+    nc += __shfl_xor_sync(0xffffffffu, nc, 1);
+    if (t < L && half == 0) {
+      const float den = fmaxf(sqrtf(na), kCosEps) * fmaxf(sqrtf(nc), kCosEps);
+      s_dis[t] = c == t ? -INFINITY : 1.f - dot / den;
+    }
   }
   __syncthreads();
 
-  // rank of each non-centre: tokens more dissimilar, or as dissimilar and earlier
+  // rank of each non-centre: tokens more dissimilar, or as dissimilar and earlier;
+  // each thread of the pair counts over one half of the block
   const int windows = (L + w - 1) / w;
   const int K = max(static_cast<int>(ceil(static_cast<double>(r) * L)), windows);
   const int extra = K - windows;
   bool kept = false;
-  if (tid < L) {
-    const float dt = s_dis[tid];
-    if (dt == -INFINITY) {
-      kept = true;
-    } else if (extra > 0) {
-      int rank = 0;
-      for (int u = 0; u < L; ++u) {
+  {
+    const float dt = t < L ? s_dis[t] : -INFINITY;
+    int rank = 0;
+    if (t < L && dt != -INFINITY && extra > 0) {
+      const int u0 = half * (kBlock / 2), u1 = min(L, u0 + kBlock / 2);
+      for (int u = u0; u < u1; ++u) {
         const float du = s_dis[u];
-        rank += (du > dt) | ((du == dt) & (u < tid));
+        rank += (du > dt) | ((du == dt) & (u < t));
       }
-      kept = rank < extra;
     }
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    kept = t < L && (dt == -INFINITY || (extra > 0 && rank < extra));
   }
-  // compact slots in position order
-  const unsigned bal = __ballot_sync(0xffffffffu, kept);
+  // compact slots in position order (one vote per token: the even thread)
+  const unsigned bal = __ballot_sync(0xffffffffu, kept && half == 0);
   if (lane == 0) s_wtot[warp] = __popc(bal);
   __syncthreads();
   int base = 0, nkept = 0;
@@ -144,15 +151,18 @@ __global__ void __launch_bounds__(kPruneThreads)
     nkept += s_wtot[k];
   }
   const int slot = base + __popc(bal & ((1u << lane) - 1u));
-  if (tid < kBlock) s_slot[tid] = kept ? slot : -1;
-  if (kept) s_tok[slot] = tid;
+  if (half == 0) {
+    s_slot[t] = kept ? slot : -1;
+    if (kept) s_tok[slot] = t;
+  }
   __syncthreads();
 
   const int S = kBlock / pack;
   const int tile = I / pack, sub = I % pack;
   const int row0 = tile * kBlock + sub * S;  // first compact row of this block
   if (tid < L) {
-    const int c = kept ? tid : centre(tid);
+    const bool kt = s_slot[tid] >= 0;
+    const int c = kt ? tid : centre(tid);
     const int64_t g = static_cast<int64_t>(bh) * N + s0 + tid;
     src_pos[g] = s0 + c;
     src_row[g] = row0 + s_slot[c];
@@ -161,11 +171,10 @@ __global__ void __launch_bounds__(kPruneThreads)
   // slots of its tile that no block owns.  16-byte pieces, kVec per row.
   const int zero_end = (I == nb - 1) ? (tile + 1) * kBlock - row0 : S;
   uint4* qs = reinterpret_cast<uint4*>(q_s + (static_cast<int64_t>(bh) * Ns + row0) * D);
-  const uint4* sq = reinterpret_cast<const uint4*>(s_q);
   for (int i = tid; i < zero_end * kVec; i += kPruneThreads) {
     const int sl = i / kVec, v = i - sl * kVec;
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (sl < nkept && sl < S) x = sq[s_tok[sl] * kVec + v];
+    if (sl < nkept && sl < S) x = s_q[piece(s_tok[sl], v)];
     qs[i] = x;
   }
 }
