@@ -599,23 +599,29 @@ def main():
         "gpu_launches": KERNELS_PER_STEP * args.steps,
     }
 
-    # ---- end to end through the public call, host buffers in and out
-    qh, kh, vh = (x[n].pin_memory() for n in ("q", "k", "v"))
+    # ---- end to end through the public host-buffer call (asa_attention_host): pinned
+    # raster Q, K, V in, raster O out, the library's copies pipelined against its
+    # kernels; device time on the caller's stream, which the call joins at both ends
+    qh, kh, vh = (x[n].contiguous().pin_memory() for n in ("q", "k", "v"))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    # device time on the launching stream, from the first H2D copy to the end of the D2H
-    e_ms = []
-    for i in range(args.e2e_steps + 2):
-        e0, e1 = ev(), ev()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
-        o_d, _, _ = asa.asa_attention(qd, kd, vd, T, Hg, W, wl.tau)
-        oh.copy_(o_d, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= 2:
-            e_ms.append(e0.elapsed_time(e1))
-    e_s = statistics.median(e_ms) * 1e-3
+    hws = asa.host_workspace(B, T, Hg, W, H, d)
+
+    def host_call_ms(reps, chunk=0, workspace=hws):
+        out = []
+        for i in range(reps + 2):
+            e0, e1 = ev(), ev()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            asa.asa_attention_host(qh, kh, vh, T, Hg, W, wl.tau, head_chunk=chunk, out=oh,
+                                   workspace=workspace, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                out.append(e0.elapsed_time(e1))
+        return statistics.median(out)
+
+    e_s = host_call_ms(args.e2e_steps) * 1e-3
+    asa.asa_check_device_status()
 
     # whole job: max over ranks of each time, work summed over ranks
     if world > 1:
@@ -627,10 +633,31 @@ def main():
     nbytes = q.numel() * q.element_size()
     result["e2e"] = {"value": total_flops / e_s / 1e12, "unit": "TFLOP/s",
                      "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
-                     "ms_per_call": e_s * 1e3, "timing": "CUDA events on the stream"}
+                     "ms_per_call": e_s * 1e3, "timing": "CUDA events on the stream",
+                     "call": "asa_attention_host (pinned host buffers, head chunks pipelined)"}
 
     if not args.no_extras:
         result["extras"] = extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream)
+        # the host-buffer call by head chunk, and the unpipelined sequence (copy Q, K, V
+        # in, device call, copy O out) for comparison
+        by_chunk = {}
+        for c in (1, 2, 3, 4, 6, 12):
+            if c <= H:
+                by_chunk[c] = host_call_ms(3, c, asa.host_workspace(B, T, Hg, W, H, d, 0, c))
+        seq = []
+        for i in range(5):
+            e0, e1 = ev(), ev()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            qd, kd, vd = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+            o_d, _, _ = asa.asa_attention(qd, kd, vd, T, Hg, W, wl.tau)
+            oh.copy_(o_d, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                seq.append(e0.elapsed_time(e1))
+        result["extras"]["host_call_ms_by_head_chunk"] = by_chunk
+        result["extras"]["host_sequential_ms"] = statistics.median(seq)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_oracle_sample(wl, x)

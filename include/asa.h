@@ -336,6 +336,37 @@ int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, 
                                int pack, int global_window, void* workspace, size_t ws_bytes,
                                void* dq, void* dk, void* dv, void* stream);
 
+/* ------------------------------------------------------------------------------
+ * One ASA (or ASA_G) self-attention call on HOST buffers: raster q, k, v in, raster O
+ * out, with the copies pipelined against the compute.
+ * ---------------------------------------------------------------------------- */
+
+/* Workspace bytes of asa_attention_host: two pipeline slots, each holding the device
+ * copies of head_chunk heads (raster and permuted Q, K, V; permuted and raster O), the
+ * estimator and mask workspace and CSR, the forward workspace and the LSE of those
+ * heads.  head_chunk = 0 takes ceil(H / 4).  0 for invalid sizes. */
+size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int d,
+                                         int global_window, int head_chunk);
+
+/*
+ * The whole call of asa_gilbert_permute3 -> asa_estimate_mask -> asa_sparse_attn_fwd
+ * -> asa_unpermute (Preprocessing, Steps 1, 2.1, 2.2) for host buffers q, k, v, o
+ * (bf16 [B, T*Hg*W, H, d], raster order), in chunks of head_chunk heads (0: ceil(H/4)).
+ * Chunk c's strided host-to-device copies, chunk c-1's kernels and chunk c-2's
+ * device-to-host copy run at once on three streams the library owns (one set per
+ * device, released by asa_shutdown); two workspace slots alternate.  The call is
+ * ordered on `stream`: the pipeline starts after the work already queued there and
+ * the stream waits for its end, so an event recorded on `stream` after the call marks
+ * the output's arrival in `o` (synchronise the stream before reading it).  Copies
+ * overlap only when the host buffers are page-locked (pinned); pageable buffers give
+ * the same results, copied synchronously.  The outputs equal asa_attention's per
+ * head: each head's mask and rows do not depend on the other heads.  Returns as the
+ * composed calls do (their argument checks apply per chunk).
+ */
+int asa_attention_host(const void* q, const void* k, const void* v, int B, int T, int Hg, int W,
+                       int H, int d, float tau, int global_window, int head_chunk,
+                       void* workspace, size_t ws_bytes, void* o, void* stream);
+
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of
  * the current device.  Returns ASA_OK, ASA_ERR_TIMEOUT if a kernel gave up a

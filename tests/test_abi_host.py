@@ -230,3 +230,30 @@ def test_prune_workspace_sizes(L):
     assert bw < L.asa_bwd_workspace_size(1, 12, N, d, 0) + BH * Ns * d * 4 + BH * 128 * 256 * 8
     assert L.asa_bwd_pruned_workspace_size(1, 12, N, 96, 2, 0) == 0
     assert L.asa_bwd_pruned_workspace_size(1, 12, N, d, 3, 0) == 0
+
+
+def test_host_call_rejects(L):
+    ws = ctypes.c_void_p(0x100000)
+    args = lambda q=FAKE, chunk=0, tau=0.9, wsb=1 << 40, T=4: (
+        q, FAKE, FAKE, 1, T, 16, 16, 2, 64, tau, 0, chunk, ws, wsb, FAKE, None)
+    assert L.asa_attention_host(*args(q=None)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_attention_host(*args(chunk=-1)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_attention_host(*args(tau=0.0)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_attention_host(*args(T=0)) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_attention_host(*args(wsb=10)) == asa.ASA_ERR_WORKSPACE
+
+
+def test_host_call_workspace_sizes(L):
+    # two slots of head_chunk heads: 8 raster/permuted tensors of B*hc*N*d bf16 each, plus
+    # the per-chunk estimator, mask and forward workspaces
+    B, T, Hg, W, H, d = 1, 21, 30, 52, 12, 128
+    N = T * Hg * W
+    one = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 1)
+    three = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 3)
+    assert three == L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0)   # ceil(12/4)
+    assert one >= 2 * 8 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
+    assert 2.5 * one < three < 3.5 * one
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 99) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, H)
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, 96, 0, 0) == 0
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, -1) == 0

@@ -53,6 +53,9 @@ _SIGNATURES = {
     "asa_sparse_attn_fwd_pruned": ([_vp] * 7 + [_c_int] * 7 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
     "asa_bwd_pruned_workspace_size": ([_c_int] * 6, _c_size),
     "asa_sparse_attn_bwd_pruned": ([_vp] * 10 + [_c_int] * 7 + [_vp, _c_size] + [_vp] * 4, _c_int),
+    "asa_attention_host_workspace_size": ([_c_int] * 8, _c_size),
+    "asa_attention_host": ([_vp] * 3 + [_c_int] * 6 + [_c_float, _c_int, _c_int, _vp, _c_size, _vp,
+                                                      _vp], _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),
@@ -490,6 +493,32 @@ def asa_attention(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: i
         op, lse = asa_sparse_attn_fwd_pruned(prune, kp, vp, tmask, global_window=global_window,
                                              stream=stream)
     return asa_unpermute(op, T, Hg, W, stream=stream), lse, mask
+
+
+def host_workspace(B, T, Hg, W, H, d, global_window=0, head_chunk=0, device="cuda"):
+    return _workspace(lib().asa_attention_host_workspace_size(B, T, Hg, W, H, d, global_window,
+                                                              head_chunk), device)
+
+
+def asa_attention_host(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
+                       head_chunk: int = 0, out=None, workspace=None, stream=None):
+    """asa_attention on host (CPU) tensors q, k, v [B, N, H, d] bf16: the library copies
+    chunks of heads in, computes and copies O out, pipelined on its own streams; pin the
+    tensors (tensor.pin_memory()) for the copies to overlap.  Returns O [B, N, H, d] on
+    the host; synchronise the stream (torch.cuda.current_stream by default) before
+    reading it."""
+    for n_, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{n_} must be a contiguous 4-D bf16 host tensor")
+    B, N, H, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if workspace is None:
+        workspace = host_workspace(B, T, Hg, W, H, d, global_window, head_chunk)
+    _check(lib().asa_attention_host(_ptr(q), _ptr(k), _ptr(v), B, T, Hg, W, H, d, float(tau),
+                                    global_window, head_chunk, _ptr(workspace),
+                                    _ws_bytes(workspace), _ptr(out), _stream(stream)))
+    return out
 
 
 class ASAAttention(torch.autograd.Function):

@@ -2,8 +2,9 @@
 //
 // Every entry point validates its arguments on the host before it launches
 // anything, carves the caller's workspace, and launches the kernels of its step on
-// the caller's stream.  The only memory the library owns is the per-shape Gilbert
-// permutation table (built on the host once per (device, T, Hg, W) and uploaded).
+// the caller's stream.  The library owns only the per-shape Gilbert permutation table
+// (built on the host once per (device, T, Hg, W) and uploaded) and, per device, the
+// three streams and the events of the pipelined host-buffer call.
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
@@ -665,6 +666,170 @@ int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, 
   return ASA_OK;
 }
 
+// ---------------------------------------------------------------- host-buffer call
+
+namespace {
+
+// Streams (copy in, compute, copy out) and events of the host-buffer call, one set per
+// device, created on first use and released by asa_shutdown.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, cmp = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+std::mutex g_pipe_mu;
+std::map<int, HostPipe> g_pipes;
+
+int host_chunk(int H, int head_chunk) {
+  return head_chunk > 0 ? std::min(head_chunk, H) : std::max(1, (H + 3) / 4);
+}
+
+// One slot of the pipeline: raster inputs, permuted inputs, permuted and raster
+// output, estimator + mask workspace and CSR, forward workspace and LSE, for hc heads.
+struct HostSlot {
+  char* x[3];
+  char* xp[3];
+  char* op;
+  char* out;
+  char* est_ws;
+  size_t est_bytes;
+  int32_t *row_ptr, *col_idx, *nnz;
+  char* fwd_ws;
+  size_t fwd_bytes;
+  float* lse;
+  size_t bytes;
+};
+
+HostSlot carve_host_slot(char* base, int B, int hc, int N, int d, int global_window) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base == nullptr ? nullptr : base + off;
+    off += align256(bytes);
+    return p;
+  };
+  HostSlot r{};
+  const size_t t = static_cast<size_t>(B) * hc * N * d * 2;
+  const size_t nb = (static_cast<size_t>(N) + ASA_BLOCK - 1) / ASA_BLOCK;
+  const size_t rows = static_cast<size_t>(B) * hc * nb;
+  for (int i = 0; i < 3; ++i) r.x[i] = take(t);
+  for (int i = 0; i < 3; ++i) r.xp[i] = take(t);
+  r.op = take(t);
+  r.out = take(t);
+  r.est_bytes = asa_estimate_mask_workspace_size(B, hc, N);
+  r.est_ws = take(r.est_bytes);
+  r.row_ptr = reinterpret_cast<int32_t*>(take((rows + 1) * 4));
+  r.col_idx = reinterpret_cast<int32_t*>(take(rows * nb * 4));
+  r.nnz = reinterpret_cast<int32_t*>(take(4));
+  r.fwd_bytes = asa_fwd_workspace_size(B, hc, N, d, global_window);
+  r.fwd_ws = take(r.fwd_bytes);
+  r.lse = reinterpret_cast<float*>(take(static_cast<size_t>(B) * hc * N * 4));
+  r.bytes = off;
+  return r;
+}
+
+}  // namespace
+
+size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int d,
+                                         int global_window, int head_chunk) {
+  const int64_t N = static_cast<int64_t>(T) * Hg * W;
+  if (B < 1 || H < 1 || T < 1 || Hg < 1 || W < 1 || N > ASA_MAX_TOKENS || (d != 64 && d != 128) ||
+      global_window < 0 || head_chunk < 0)
+    return 0;
+  const int hc = host_chunk(H, head_chunk);
+  return 2 * carve_host_slot(nullptr, B, hc, static_cast<int>(N), d, global_window).bytes;
+}
+
+int asa_attention_host(const void* q, const void* k, const void* v, int B, int T, int Hg, int W,
+                       int H, int d, float tau, int global_window, int head_chunk,
+                       void* workspace, size_t ws_bytes, void* o, void* stream) {
+  int64_t N64 = 0;
+  ASA_TRY(check_grid(T, Hg, W, &N64));
+  const int N = static_cast<int>(N64);
+  ASA_TRY(check_common(B, H, N, d));
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
+    return fail(ASA_ERR_INVALID_ARG, "a host buffer (q, k, v or o) is NULL");
+  if (head_chunk < 0) return fail(ASA_ERR_INVALID_ARG, "head_chunk=%d < 0", head_chunk);
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  if (!(tau > 0.f)) return fail(ASA_ERR_INVALID_ARG, "tau=%g must be > 0", tau);
+  ASA_TRY(check_ws(workspace, ws_bytes,
+                   asa_attention_host_workspace_size(B, T, Hg, W, H, d, global_window, head_chunk)));
+  const int hc = host_chunk(H, head_chunk);
+  const int nch = (H + hc - 1) / hc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& P = g_pipes[dev];
+  if (P.h2d == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&P.cmp, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "stream creation");
+  }
+  const size_t need_ev = 4 + 3 * static_cast<size_t>(nch);
+  while (P.ev.size() < need_ev) {
+    cudaEvent_t ev;
+    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "event creation");
+    P.ev.push_back(ev);
+  }
+  cudaStream_t caller = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev_start = P.ev[0];
+  auto h2d_done = [&](int c) { return P.ev[4 + 3 * c]; };
+  auto cmp_done = [&](int c) { return P.ev[5 + 3 * c]; };
+  auto d2h_done = [&](int c) { return P.ev[6 + 3 * c]; };
+  // on any failure after work was enqueued: the caller's stream still waits for it
+  auto finish = [&](int rc) {
+    cudaEventRecord(P.ev[1], P.h2d);
+    cudaEventRecord(P.ev[2], P.cmp);
+    cudaEventRecord(P.ev[3], P.d2h);
+    for (int i = 1; i <= 3; ++i) cudaStreamWaitEvent(caller, P.ev[i], 0);
+    return rc;
+  };
+  if ((e = cudaEventRecord(ev_start, caller)) != cudaSuccess) return cuda_fail(e, "event record");
+  for (cudaStream_t s : {P.h2d, P.cmp, P.d2h}) cudaStreamWaitEvent(s, ev_start, 0);
+
+  const size_t slot_bytes = carve_host_slot(nullptr, B, hc, N, d, global_window).bytes;
+  const size_t pitch = static_cast<size_t>(H) * d * 2;
+  const void* src[3] = {q, k, v};
+  for (int c = 0; c < nch; ++c) {
+    const HostSlot S = carve_host_slot(static_cast<char*>(workspace) + (c & 1) * slot_bytes, B, hc,
+                                       N, d, global_window);
+    const int h0 = c * hc, hcur = std::min(hc, H - h0);
+    const size_t width = static_cast<size_t>(hcur) * d * 2;
+    // copy in: the slot's inputs are free once chunk c - 2 has been computed
+    if (c >= 2) cudaStreamWaitEvent(P.h2d, cmp_done(c - 2), 0);
+    for (int i = 0; i < 3; ++i) {
+      e = cudaMemcpy2DAsync(S.x[i], width, static_cast<const char*>(src[i]) + h0 * d * 2, pitch,
+                            width, static_cast<size_t>(B) * N, cudaMemcpyHostToDevice, P.h2d);
+      if (e != cudaSuccess) return finish(cuda_fail(e, "host-to-device copy"));
+    }
+    cudaEventRecord(h2d_done(c), P.h2d);
+    // compute: the slot's output is free once chunk c - 2 has been copied out
+    cudaStreamWaitEvent(P.cmp, h2d_done(c), 0);
+    if (c >= 2) cudaStreamWaitEvent(P.cmp, d2h_done(c - 2), 0);
+    int rc = asa_gilbert_permute3(S.x[0], S.x[1], S.x[2], S.xp[0], S.xp[1], S.xp[2], B, T, Hg, W,
+                                  hcur, d, P.cmp);
+    if (rc == ASA_OK)
+      rc = asa_estimate_mask(S.xp[0], S.xp[1], B, hcur, N, d, ASA_BLOCK, ASA_SAMPLES, tau, S.est_ws,
+                             S.est_bytes, S.row_ptr, S.col_idx, S.nnz, nullptr, nullptr, P.cmp);
+    if (rc == ASA_OK)
+      rc = asa_sparse_attn_fwd(S.xp[0], S.xp[1], S.xp[2], S.row_ptr, S.col_idx, B, hcur, N, d,
+                               ASA_BLOCK, global_window, S.fwd_ws, S.fwd_bytes, S.op, S.lse, P.cmp);
+    if (rc == ASA_OK) rc = asa_unpermute(S.op, S.out, B, T, Hg, W, hcur, d, P.cmp);
+    if (rc != ASA_OK) return finish(rc);
+    cudaEventRecord(cmp_done(c), P.cmp);
+    // copy out
+    cudaStreamWaitEvent(P.d2h, cmp_done(c), 0);
+    e = cudaMemcpy2DAsync(static_cast<char*>(o) + h0 * d * 2, pitch, S.out, width, width,
+                          static_cast<size_t>(B) * N, cudaMemcpyDeviceToHost, P.d2h);
+    if (e != cudaSuccess) return finish(cuda_fail(e, "device-to-host copy"));
+    cudaEventRecord(d2h_done(c), P.d2h);
+  }
+  if ((e = cudaStreamWaitEvent(caller, d2h_done(nch - 1), 0)) != cudaSuccess)
+    return finish(cuda_fail(e, "stream wait"));
+  return ASA_OK;
+}
+
 int asa_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1 || limit_cycles > (1ll << 31))
     return fail(ASA_ERR_INVALID_ARG, "limit_cycles=%lld outside [1, 2^31]", limit_cycles);
@@ -698,6 +863,22 @@ int asa_check_device_status(void* stream) {
 }
 
 void asa_shutdown(void) {
+  {
+    std::lock_guard<std::mutex> plock(g_pipe_mu);
+    int cur = 0;
+    const bool have = cudaGetDevice(&cur) == cudaSuccess;
+    for (auto& kv : g_pipes) {
+      if (have) cudaSetDevice(kv.first);
+      for (cudaStream_t s : {kv.second.h2d, kv.second.cmp, kv.second.d2h})
+        if (s != nullptr) {
+          cudaStreamSynchronize(s);
+          cudaStreamDestroy(s);
+        }
+      for (cudaEvent_t ev : kv.second.ev) cudaEventDestroy(ev);
+    }
+    if (have) cudaSetDevice(cur);
+    g_pipes.clear();
+  }
   std::lock_guard<std::mutex> lock(g_perm_mu);
   int cur = 0;
   const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
