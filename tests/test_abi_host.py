@@ -250,7 +250,9 @@ def test_host_call_workspace_sizes(L):
     N = T * Hg * W
     one = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 1)
     three = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 3)
-    assert three == L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0)   # ceil(12/4)
+    assert one == L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0)     # ceil(12/12)
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 0) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 4)               # ceil(48/12)
     assert one >= 2 * 8 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
     assert 2.5 * one < three < 3.5 * one
     assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 99) == \

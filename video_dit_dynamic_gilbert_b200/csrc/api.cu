@@ -680,7 +680,7 @@ std::mutex g_pipe_mu;
 std::map<int, HostPipe> g_pipes;
 
 int host_chunk(int H, int head_chunk) {
-  return head_chunk > 0 ? std::min(head_chunk, H) : std::max(1, (H + 3) / 4);
+  return head_chunk > 0 ? std::min(head_chunk, H) : std::max(1, (H + 11) / 12);
 }
 
 // One slot of the pipeline: raster inputs, permuted inputs, permuted and raster
