@@ -313,31 +313,32 @@ __global__ void __launch_bounds__(256)
 // Backward inputs in the compact layout: for a kept token i (src_pos[i] = i) with
 // compact row r = src_row[i], dO'_s[r] = the sum of dO[j] over the tokens j of i's
 // block with src_pos[j] = i (its own gradient and those of the pruned tokens it
-// fills), stored in bf16, and lse2_s[r] = lse[i] log2(e).  One warp per token; a
-// pruned token only checks that it points at a kept token of its own block.
+// fills), stored in bf16, and lse2_s[r] = lse[i] log2(e).  One CTA per (b, h, block):
+// the block's src_pos is staged in shared memory (every token is checked to point at
+// a kept token of its own block); each warp then takes kept tokens and finds their
+// contributors with four ballots over shared memory.
 template <int D>
 __global__ void __launch_bounds__(256)
     dout_compact_kernel(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                         const int32_t* __restrict__ src_pos, const int32_t* __restrict__ src_row,
-                        int64_t rows, int N, int Ns, __nv_bfloat16* __restrict__ dout_s,
+                        int N, int nb, int Ns, __nv_bfloat16* __restrict__ dout_s,
                         float* __restrict__ lse2_s, unsigned int* __restrict__ err_word) {
   constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       row < rows; row += warps) {
-    const int64_t bh = row / N;
-    const int i = static_cast<int>(row - bh * N);
-    const int s0 = (i / kBlock) * kBlock;
-    const int L = min(kBlock, N - s0);
-    const int32_t* sp = src_pos + bh * N;
-    const int p = sp[i];
-    if (p != i) {
-      const bool bad = p < s0 || p >= s0 + L || sp[p] != p;
-      if (bad && lane == 0) atomicOr(err_word, kErrBadIndex);
-      continue;
-    }
-    const int r = src_row[row];
+  __shared__ int s_sp[kBlock];
+  const int bh = blockIdx.x / nb, I = blockIdx.x % nb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int s0 = I * kBlock;
+  const int L = min(kBlock, N - s0);
+  const int64_t g0 = static_cast<int64_t>(bh) * N + s0;  // first token of the block
+  if (tid < L) s_sp[tid] = src_pos[g0 + tid] - s0;       // block-relative source
+  __syncthreads();
+  if (tid < L) {
+    const int p = s_sp[tid];
+    if (p < 0 || p >= L || s_sp[p] != p) atomicOr(err_word, kErrBadIndex);
+  }
+  for (int t = warp; t < L; t += 8) {
+    if (s_sp[t] != t) continue;  // pruned: its gradient goes to its source
+    const int r = src_row[g0 + t];
     if (r < 0 || r >= Ns) {
       if (lane == 0) atomicOr(err_word, kErrBadIndex);
       continue;
@@ -345,25 +346,26 @@ __global__ void __launch_bounds__(256)
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int j0 = 0; j0 < L; j0 += 32) {
+#pragma unroll
+    for (int j0 = 0; j0 < kBlock; j0 += 32) {
       const int j = j0 + lane;
-      unsigned m = __ballot_sync(0xffffffffu, j < L && sp[s0 + j] == i);
+      unsigned m = __ballot_sync(0xffffffffu, j < L && s_sp[j] == t);
       while (m != 0u) {
         const int b = __ffs(m) - 1;
         m &= m - 1u;
         float x[E];
-        load_bf16<E>(dout + (bh * N + s0 + j0 + b) * D + lane * E, x);
+        load_bf16<E>(dout + (g0 + j0 + b) * D + lane * E, x);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] += x[e];
       }
     }
-    __nv_bfloat16* dst = dout_s + (bh * Ns + r) * D + lane * E;
+    __nv_bfloat16* dst = dout_s + (static_cast<int64_t>(bh) * Ns + r) * D + lane * E;
     if constexpr (E == 4) {
       *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
     } else {
       *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0], acc[1]);
     }
-    if (lane == 0) lse2_s[bh * Ns + r] = lse[row] * kLog2e;
+    if (lane == 0) lse2_s[static_cast<int64_t>(bh) * Ns + r] = lse[g0 + t] * kLog2e;
   }
 }
 
@@ -506,16 +508,16 @@ cudaError_t launch_dout_compact(const void* dout, const float* lse, const int32_
                                 const int32_t* src_row, int BH, int N, int Ns, int d,
                                 void* dout_s, float* lse2_s, unsigned int* err_word, int num_sms,
                                 cudaStream_t stream) {
-  const int64_t rows = static_cast<int64_t>(BH) * N;
-  const unsigned grid = grid_of(rows, 8, num_sms, 8);
+  const int nb = (N + kBlock - 1) / kBlock;
   const auto* src = static_cast<const __nv_bfloat16*>(dout);
   auto* dst = static_cast<__nv_bfloat16*>(dout_s);
   if (d == 128)
-    dout_compact_kernel<128><<<grid, 256, 0, stream>>>(src, lse, src_pos, src_row, rows, N, Ns, dst,
-                                                       lse2_s, err_word);
+    dout_compact_kernel<128><<<BH * nb, 256, 0, stream>>>(src, lse, src_pos, src_row, N, nb, Ns,
+                                                          dst, lse2_s, err_word);
   else
-    dout_compact_kernel<64><<<grid, 256, 0, stream>>>(src, lse, src_pos, src_row, rows, N, Ns, dst,
-                                                      lse2_s, err_word);
+    dout_compact_kernel<64><<<BH * nb, 256, 0, stream>>>(src, lse, src_pos, src_row, N, nb, Ns,
+                                                         dst, lse2_s, err_word);
+  (void)num_sms;
   return cudaGetLastError();
 }
 
