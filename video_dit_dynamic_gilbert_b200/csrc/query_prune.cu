@@ -314,9 +314,10 @@ __global__ void __launch_bounds__(256)
 // compact row r = src_row[i], dO'_s[r] = the sum of dO[j] over the tokens j of i's
 // block with src_pos[j] = i (its own gradient and those of the pruned tokens it
 // fills), stored in bf16, and lse2_s[r] = lse[i] log2(e).  One CTA per (b, h, block):
-// the block's src_pos is staged in shared memory (every token is checked to point at
-// a kept token of its own block); each warp then takes kept tokens and finds their
-// contributors with four ballots over shared memory.
+// the block's src_pos and dO rows are staged in shared memory (every load in flight
+// before the stores; every token is checked to point at a kept token of its own
+// block); each warp then takes kept tokens, finds their contributors with four
+// ballots and sums their rows from shared memory.
 template <int D>
 __global__ void __launch_bounds__(256)
     dout_compact_kernel(const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
@@ -324,12 +325,30 @@ __global__ void __launch_bounds__(256)
                         int N, int nb, int Ns, __nv_bfloat16* __restrict__ dout_s,
                         float* __restrict__ lse2_s, unsigned int* __restrict__ err_word) {
   constexpr int E = D / 32;
+  constexpr int kVec = D / 8;  // 16-byte pieces per row
+  __shared__ __align__(16) __nv_bfloat16 s_do[kBlock * D];
   __shared__ int s_sp[kBlock];
   const int bh = blockIdx.x / nb, I = blockIdx.x % nb;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s0 = I * kBlock;
   const int L = min(kBlock, N - s0);
   const int64_t g0 = static_cast<int64_t>(bh) * N + s0;  // first token of the block
+  {
+    constexpr int kPer = kBlock * kVec / 256;
+    const uint4* src = reinterpret_cast<const uint4*>(dout + g0 * D);
+    uint4* dst = reinterpret_cast<uint4*>(s_do);
+    uint4 v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * 256;
+      if (i < L * kVec) v[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * 256;
+      if (i < L * kVec) dst[i] = v[u];
+    }
+  }
   if (tid < L) s_sp[tid] = src_pos[g0 + tid] - s0;       // block-relative source
   __syncthreads();
   if (tid < L) {
@@ -354,7 +373,7 @@ __global__ void __launch_bounds__(256)
         const int b = __ffs(m) - 1;
         m &= m - 1u;
         float x[E];
-        load_bf16<E>(dout + (g0 + j0 + b) * D + lane * E, x);
+        load_bf16<E>(s_do + (j0 + b) * D + lane * E, x);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] += x[e];
       }
