@@ -403,6 +403,47 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
     return r, (qp, kp, vp)
 
 
+def _seqpar_stages(asa, torch, timer, wl, dev, peaks, P=8):
+    """The sequence-parallel local steps of rank 0 of P ranks emulated on this GPU (the
+    all-to-alls are replaced by slicing): pack of its token shard, the Gilbert gather
+    from its receive chunks, the inverse into its send chunks, the unpack."""
+    from inputs import make_inputs
+    from video_dit_dynamic_gilbert_b200 import seqpar
+    x = make_inputs(wl)
+    full = [x[n].to(dev) for n in ("q", "k", "v")]
+    B, N, H, d = full[0].shape
+    T, Hg, W = wl.T, wl.Hg, wl.W
+    tok, heads = seqpar.shard_offsets(N, P), seqpar.shard_offsets(H, P)
+    ops = seqpar.KernelOps()
+    Hl, N0 = heads[1] - heads[0], tok[1] - tok[0]
+    shard0 = [t[:, tok[0]:tok[1]].contiguous() for t in full]
+    recv0 = []
+    for t in full:        # rank 0's receive buffer: every rank's tokens of heads [0, Hl)
+        recv0.append(torch.cat([t[:, tok[s]:tok[s + 1], heads[0]:heads[1]].reshape(-1)
+                                for s in range(P)]))
+    op0 = torch.randn((B, Hl, N, d), device=dev).to(torch.bfloat16)
+    back0 = torch.cat([full[0][:, tok[0]:tok[1], heads[s]:heads[s + 1]].reshape(-1)
+                       for s in range(P)])
+    hbm = peaks[2]
+    r = {"P": P, "rank0_tokens": N0, "rank0_heads": Hl}
+
+    def stage(name, fn, nbytes):
+        t = timer(fn)
+        t["GB_s"] = nbytes / (t["median_ms"] * 1e-3) / 1e9
+        t["frac_of_measured_hbm"] = t["GB_s"] / hbm
+        r[name] = t
+
+    shard_bytes = B * N0 * H * d * 2
+    recv_bytes = B * N * Hl * d * 2
+    stage("pack_q", lambda: ops.pack(shard0[0], heads), 2 * shard_bytes)
+    stage("permute3_from_chunks", lambda: ops.permute3(recv0, tok, B, T, Hg, W, Hl, d),
+          3 * 2 * recv_bytes)
+    stage("unpermute_to_chunks", lambda: ops.unpermute(op0, tok, T, Hg, W), 2 * recv_bytes)
+    stage("unpack_o", lambda: ops.unpack(back0, heads, (B, N0, H, d)), 2 * shard_bytes)
+    asa.asa_check_device_status()
+    return r
+
+
 def _dense(asa, torch, timer, qp, kp, vp, peaks):
     """Dense attention on the same inputs: our kernel with every tile kept, and torch SDPA."""
     B, H, N, d = qp.shape
@@ -460,6 +501,8 @@ def run_report(path):
                     "estimate_mask_share": em["median_ms"] / (em["median_ms"] + fw["median_ms"])})
         del qp, kp, vp
         torch.cuda.empty_cache()
+    rep["seqpar_emulated"] = {"wan-14b-720p": _seqpar_stages(asa, torch, timer,
+                                                             WORKLOADS["wan-14b-720p"], dev, peaks)}
     rep["clocks"] = clocks.stop()
     with open(path, "w") as f:
         json.dump(rep, f, indent=1)
@@ -478,6 +521,10 @@ def run_report(path):
         if "attn_bwd" in qpr:
             line += f" bwd {qpr['attn_bwd']['median_ms']:.2f} ms (x{qpr['bwd_speedup']:.2f})"
         print(line)
+    for name, sp in rep["seqpar_emulated"].items():
+        print(f"{name} seqpar rank 0 of {sp['P']}: " + ", ".join(
+            f"{k} {sp[k]['median_ms']:.3f} ms {sp[k]['GB_s']:.0f} GB/s" for k in
+            ("pack_q", "permute3_from_chunks", "unpermute_to_chunks", "unpack_o")))
     return rep
 
 

@@ -52,6 +52,7 @@ extern "C" {
 
 #define ASA_MAX_TOKENS 262144   /* N limit: at most 2048 blocks of 128 */
 #define ASA_BLOCK 128
+#define ASA_MAX_RANKS 64       /* sequence-parallel ranks of the asa_seqpar_* calls */
 #define ASA_SAMPLES 16
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -367,6 +368,44 @@ size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int
 int asa_attention_host(const void* q, const void* k, const void* v, int B, int T, int Hg, int W,
                        int H, int d, float tau, int global_window, int head_chunk,
                        void* workspace, size_t ws_bytes, void* o, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Sequence parallelism (a sequence-sharded DiT): P ranks, rank r holding the raster
+ * tokens [tok_off[r], tok_off[r+1]) of every head, x_r [B, N_r, H, d].  Attention
+ * needs every token of a head, so before it an all-to-all (NCCL, into local buffers)
+ * gives rank r every token of its heads [head_off[r], head_off[r+1]), H_r of them;
+ * the inverse all-to-all follows.  These calls are the local steps around the two
+ * exchanges; the Gilbert gather reads the receive buffer's per-rank chunks directly
+ * and the inverse writes straight into the send buffer's chunks.  Offsets are host
+ * arrays of P + 1 ints from 0 to N (tokens) or H (heads), non-decreasing;
+ * 1 <= P <= ASA_MAX_RANKS.  Device buffers bf16, 16-byte aligned.
+ * ---------------------------------------------------------------------------- */
+
+/* Send buffer of the first exchange: send = chunks s = 0..P-1 back to back, chunk s =
+ * x[:, :, head_off[s]:head_off[s+1], :] as [B, Nr, H_s, d] (for rank s).  x: [B, Nr, H, d]. */
+int asa_seqpar_pack(const void* x, void* send, int B, int Nr, int H, int d, const int* head_off,
+                    int P, void* stream);
+
+/* Inverse of asa_seqpar_pack, applied to the receive buffer of the second exchange:
+ * chunk s (from rank s, its heads) back into x [B, Nr, H, d]. */
+int asa_seqpar_unpack(const void* recv, void* x, int B, int Nr, int H, int d, const int* head_off,
+                      int P, void* stream);
+
+/*
+ * Preprocessing on the receive buffers of the first exchange: r = chunks s = 0..P-1
+ * back to back, chunk s = rank s's tokens of this rank's Hl heads as [B, N_s, Hl, d];
+ * xp[b, h, i, :] = the row of token perm[i] (Gilbert order of the T x Hg x W grid)
+ * taken from its rank's chunk.  xp: [B, Hl, N, d]; three tensors (Q, K, V) at once.
+ * With P = 1 it is asa_gilbert_permute3.
+ */
+int asa_seqpar_permute3(const void* r0, const void* r1, const void* r2, void* xp0, void* xp1,
+                        void* xp2, int B, int T, int Hg, int W, int Hl, int d, const int* tok_off,
+                        int P, void* stream);
+
+/* Inverse of asa_seqpar_permute3 for one tensor: op [B, Hl, N, d] (permuted) into the
+ * send buffer of the second exchange, chunk s = rank s's tokens [B, N_s, Hl, d]. */
+int asa_seqpar_unpermute(const void* op, void* send, int B, int T, int Hg, int W, int Hl, int d,
+                         const int* tok_off, int P, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error word of

@@ -259,3 +259,22 @@ def test_host_call_workspace_sizes(L):
         L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, H)
     assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, 96, 0, 0) == 0
     assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, -1) == 0
+
+
+def test_seqpar_rejects(L):
+    offs = lambda *v: (ctypes.c_int * len(v))(*v)
+    ok_heads = offs(0, 2, 4)
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 64, offs(0, 2, 5), 2, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 64, offs(1, 2, 4), 2, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 64, offs(0, 3, 2, 4), 3, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 64, ok_heads, 0, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 64, None, 2, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_unpack(MIS, FAKE, 1, 10, 4, 64, ok_heads, 2, None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_pack(FAKE, FAKE, 1, 10, 4, 96, ok_heads, 2, None) == asa.ASA_ERR_UNSUPPORTED
+    # token offsets must run from 0 to T*Hg*W (here 4*16*16 = 1024)
+    assert L.asa_seqpar_permute3(*([FAKE] * 6), 1, 4, 16, 16, 2, 64, offs(0, 500, 1000), 2,
+                                 None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_unpermute(FAKE, FAKE, 1, 4, 16, 16, 2, 64, offs(0, 600, 500, 1024), 3,
+                                  None) == asa.ASA_ERR_INVALID_ARG
+    assert L.asa_seqpar_unpermute(FAKE, FAKE, 1, 0, 16, 16, 2, 64, offs(0, 1024), 1,
+                                  None) == asa.ASA_ERR_INVALID_ARG

@@ -56,6 +56,10 @@ _SIGNATURES = {
     "asa_attention_host_workspace_size": ([_c_int] * 8, _c_size),
     "asa_attention_host": ([_vp] * 3 + [_c_int] * 6 + [_c_float, _c_int, _c_int, _vp, _c_size, _vp,
                                                       _vp], _c_int),
+    "asa_seqpar_pack": ([_vp, _vp] + [_c_int] * 4 + [_vp, _c_int, _vp], _c_int),
+    "asa_seqpar_unpack": ([_vp, _vp] + [_c_int] * 4 + [_vp, _c_int, _vp], _c_int),
+    "asa_seqpar_permute3": ([_vp] * 6 + [_c_int] * 6 + [_vp, _c_int, _vp], _c_int),
+    "asa_seqpar_unpermute": ([_vp, _vp] + [_c_int] * 6 + [_vp, _c_int, _vp], _c_int),
     "asa_check_device_status": ([_vp], _c_int),
     "asa_selftest_wait_timeout": ([ctypes.c_longlong, _vp], _c_int),
     "asa_shutdown": ([], None),

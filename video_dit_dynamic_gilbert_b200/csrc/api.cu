@@ -830,6 +830,91 @@ int asa_attention_host(const void* q, const void* k, const void* v, int B, int T
   return ASA_OK;
 }
 
+// ---------------------------------------------------------------- sequence parallelism
+
+namespace {
+
+// P + 1 offsets from 0 to total, non-decreasing, P in [1, ASA_MAX_RANKS]
+int check_segs(const int* off, int P, int total, const char* what, asa::Segs* out) {
+  if (off == nullptr) return fail(ASA_ERR_INVALID_ARG, "%s offsets are NULL", what);
+  if (P < 1 || P > ASA_MAX_RANKS)
+    return fail(ASA_ERR_INVALID_ARG, "P=%d ranks not in [1, %d]", P, ASA_MAX_RANKS);
+  if (off[0] != 0 || off[P] != total)
+    return fail(ASA_ERR_INVALID_ARG, "%s offsets must run from 0 to %d", what, total);
+  out->P = P;
+  for (int s = 0; s <= P; ++s) {
+    if (s > 0 && off[s] < off[s - 1])
+      return fail(ASA_ERR_INVALID_ARG, "%s offsets decrease at rank %d", what, s);
+    out->off[s] = off[s];
+  }
+  return ASA_OK;
+}
+
+}  // namespace
+
+int asa_seqpar_pack(const void* x, void* send, int B, int Nr, int H, int d, const int* head_off,
+                    int P, void* stream) {
+  ASA_TRY(check_common(B, H, std::max(Nr, 1), d));
+  if (Nr < 0) return fail(ASA_ERR_INVALID_ARG, "Nr=%d < 0", Nr);
+  ASA_TRY(check_ptr(x, "x"));
+  ASA_TRY(check_ptr(send, "send"));
+  asa::Segs heads{};
+  ASA_TRY(check_segs(head_off, P, H, "head", &heads));
+  if (Nr == 0) return ASA_OK;
+  cudaError_t e = asa::launch_head_groups(x, send, true, B, Nr, H, d, heads, num_sms_current(),
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ASA_OK : cuda_fail(e, "pack launch");
+}
+
+int asa_seqpar_unpack(const void* recv, void* x, int B, int Nr, int H, int d, const int* head_off,
+                      int P, void* stream) {
+  ASA_TRY(check_common(B, H, std::max(Nr, 1), d));
+  if (Nr < 0) return fail(ASA_ERR_INVALID_ARG, "Nr=%d < 0", Nr);
+  ASA_TRY(check_ptr(recv, "recv"));
+  ASA_TRY(check_ptr(x, "x"));
+  asa::Segs heads{};
+  ASA_TRY(check_segs(head_off, P, H, "head", &heads));
+  if (Nr == 0) return ASA_OK;
+  cudaError_t e = asa::launch_head_groups(recv, x, false, B, Nr, H, d, heads, num_sms_current(),
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ASA_OK : cuda_fail(e, "unpack launch");
+}
+
+static int seqpar_permute_impl(const void* const* src, void* const* dst, int nt, bool to_perm,
+                               int B, int T, int Hg, int W, int Hl, int d, const int* tok_off,
+                               int P, void* stream) {
+  int64_t N = 0;
+  ASA_TRY(check_grid(T, Hg, W, &N));
+  ASA_TRY(check_common(B, Hl, static_cast<int>(N), d));
+  for (int k = 0; k < nt; ++k) {
+    ASA_TRY(check_ptr(src[k], "src"));
+    ASA_TRY(check_ptr(dst[k], "dst"));
+  }
+  asa::Segs tok{};
+  ASA_TRY(check_segs(tok_off, P, static_cast<int>(N), "token", &tok));
+  const int32_t* perm = nullptr;
+  ASA_TRY(get_perm(T, Hg, W, &perm));
+  cudaError_t e = asa::launch_permute_chunks(src, dst, nt, to_perm, perm, B, static_cast<int>(N),
+                                             Hl, d, tok, num_sms_current(),
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ASA_OK : cuda_fail(e, "chunk permute launch");
+}
+
+int asa_seqpar_permute3(const void* r0, const void* r1, const void* r2, void* xp0, void* xp1,
+                        void* xp2, int B, int T, int Hg, int W, int Hl, int d, const int* tok_off,
+                        int P, void* stream) {
+  const void* s[3] = {r0, r1, r2};
+  void* t[3] = {xp0, xp1, xp2};
+  return seqpar_permute_impl(s, t, 3, true, B, T, Hg, W, Hl, d, tok_off, P, stream);
+}
+
+int asa_seqpar_unpermute(const void* op, void* send, int B, int T, int Hg, int W, int Hl, int d,
+                         const int* tok_off, int P, void* stream) {
+  const void* s[1] = {op};
+  void* t[1] = {send};
+  return seqpar_permute_impl(s, t, 1, false, B, T, Hg, W, Hl, d, tok_off, P, stream);
+}
+
 int asa_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1 || limit_cycles > (1ll << 31))
     return fail(ASA_ERR_INVALID_ARG, "limit_cycles=%lld outside [1, 2^31]", limit_cycles);

@@ -16,6 +16,14 @@ constexpr unsigned int kErrBadIndex = 32u;
 
 bool gilbert_order_host(int T, int Hg, int W, int32_t* out);
 
+// Sequence parallelism: P ranks, rank s owning the items [off[s], off[s+1]) (tokens or
+// heads); passed to kernels by value.
+constexpr int kMaxRanks = 64;
+struct Segs {
+  int P;
+  int off[kMaxRanks + 1];
+};
+
 // Records the calling thread's error message for asa_last_error_string(); returns code.
 int record_error(int code, const char* fmt, ...);
 
@@ -68,6 +76,16 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk,
                           void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream);
+
+// Gilbert gather from / scatter into per-rank token chunks: chunk s holds the rows
+// [B][tok.off[s+1] - tok.off[s]][H][d] of rank s's tokens, chunks back to back (the
+// layout of an all-to-all receive or send buffer).
+cudaError_t launch_permute_chunks(const void* const* src, void* const* dst, int ntensors,
+                                  bool to_permuted, const int32_t* perm_dev, int B, int N, int H,
+                                  int d, const Segs& tok, int num_sms, cudaStream_t stream);
+// Head groups: x [B][Nr][H][d] <-> chunks [P][B][Nr][heads of group s][d].
+cudaError_t launch_head_groups(const void* src, void* dst, bool pack, int B, int Nr, int H, int d,
+                               const Segs& heads, int num_sms, cudaStream_t stream);
 
 // Exclusive scan of n int32 counts on one CTA: out[i] = sum_{k<i} in[k], out[n] and
 // *total (if non-null) = the sum.
