@@ -94,6 +94,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
+@pytest.mark.timeout(300)
 def test_nccl_single_rank_harness():
     wl = BASE.with_(name="sp1", B=1, H=3, d=64, T=3, Hg=9, W=11, seed=63)
     x = make_inputs(wl)

@@ -78,6 +78,7 @@ def _rank(rank, world, port, T, Hg, W, H, B, d, q):
         dist.destroy_process_group()
 
 
+@pytest.mark.timeout(300)
 @pytest.mark.parametrize("world,T,Hg,W,H", [(2, 3, 5, 7, 4), (2, 2, 4, 5, 3), (3, 2, 3, 5, 5)])
 def test_seqpar_exchange_round_trip(world, T, Hg, W, H):
     ctx = mp.get_context("spawn")
