@@ -84,14 +84,19 @@ def test_seqpar_exchange_round_trip(world, T, Hg, W, H):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, T, Hg, W, H, 2, 8, q))
+    procs = [ctx.Process(target=_rank, args=(r, world, port, T, Hg, W, H, 2, 8, q), daemon=True)
              for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=120) for _ in procs]
-    for p in procs:
-        p.join(timeout=60)
-        assert p.exitcode == 0
+    try:
+        res = [q.get(timeout=120) for _ in procs]
+        for p in procs:
+            p.join(timeout=60)
+            assert p.exitcode == 0
+    finally:
+        for p in procs:          # the children this test started, if one is left waiting
+            if p.is_alive():
+                p.kill()
     N = T * Hg * W
     tok = seqpar.shard_offsets(N, world)
     for rank, ok, shape in res:
