@@ -743,6 +743,8 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
     o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, tmask)
     dout = torch.randn_like(qp)
     bwd_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, tmask), reps=5)
+    bwd_dfo_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, tmask,
+                                                        d_from_o=True), reps=5)
     flops, _, _ = _kept_tile_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
                                    B, H, N, d)
     # ASA_G backward (n = 64) on the same mask
@@ -785,6 +787,7 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
         "asa_g_fwd_ms_n64": g_ms,
         "asa_g_fwd_tflops": (flops + 4 * d * N * G * B * H) / g_ms / 1e9,
         "bwd_ms": bwd_ms, "bwd_tflops": 2.5 * flops / bwd_ms / 1e9,
+        "bwd_d_from_o_ms": bwd_dfo_ms, "bwd_d_from_o_tflops": 2.5 * flops / bwd_dfo_ms / 1e9,
         "asa_g_bwd_ms_n64": bwd_g_ms,
         "asa_g_bwd_tflops": 2.5 * (flops + 4 * d * N * G * B * H) / bwd_g_ms / 1e9,
     }

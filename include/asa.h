@@ -217,7 +217,8 @@ size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window);
  * the window's row count (its bf16 rounding passes gradients unchanged).
  * D equals rowsum(dO * O) in exact arithmetic; it is recomputed in fp32 from the kept
  * tiles because the bf16-rounded O would cost ~4e-3 relative L2 on dQ.  `o` is
- * validated but not read.  dS enters the dQ and dK products in fp16 (so do Q and K,
+ * validated but not read (asa_sparse_attn_bwd_d_from_o reads it instead of the exact
+ * D pass).  dS enters the dQ and dK products in fp16 (so do Q and K,
  * as fp16 copies in the workspace): Q and K magnitudes must stay at or below 65504;
  * a larger value is reported by the next asa_check_device_status as
  * ASA_ERR_INVALID_ARG (the gradients of that call are then meaningless).
@@ -232,6 +233,21 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
                         const int32_t* row_idx_t, int B, int H, int N, int d, int block,
                         int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
                         void* dv, void* stream);
+
+/*
+ * asa_sparse_attn_bwd with D taken as rowsum(dO * O) from the forward's bf16 O (read
+ * here) instead of the exact pass over the kept tiles: one GEMM pair per kept tile
+ * less, about a fifth of the backward's time.  The rounding of O to bf16 then enters
+ * dS: on the parity cases it adds about 3e-3 relative L2 to dQ and dK (dV does not
+ * depend on D and is bit-identical to asa_sparse_attn_bwd's).  Same arguments,
+ * workspace and errors as asa_sparse_attn_bwd; opt in where that accuracy suffices.
+ */
+int asa_sparse_attn_bwd_d_from_o(const void* qp, const void* kp, const void* vp, const void* o,
+                                 const void* dout, const float* lse, const int32_t* row_ptr,
+                                 const int32_t* col_idx, const int32_t* col_ptr_t,
+                                 const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                                 int global_window, void* workspace, size_t ws_bytes, void* dq,
+                                 void* dk, void* dv, void* stream);
 
 /* ------------------------------------------------------------------------------
  * Query pruning with token filling ("Bidirectional Sparse Attention for Faster

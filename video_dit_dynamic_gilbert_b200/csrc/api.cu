@@ -436,12 +436,11 @@ size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window) {
   return asa::bwd_tc_workspace_bytes(B * H, N, d, global_window);
 }
 
-int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
-                        const void* dout, const float* lse, const int32_t* row_ptr,
-                        const int32_t* col_idx, const int32_t* col_ptr_t,
-                        const int32_t* row_idx_t, int B, int H, int N, int d, int block,
-                        int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
-                        void* dv, void* stream) {
+static int bwd_impl(const void* qp, const void* kp, const void* vp, const void* o,
+                    const void* dout, const float* lse, const int32_t* row_ptr,
+                    const int32_t* col_idx, const int32_t* col_ptr_t, const int32_t* row_idx_t,
+                    int B, int H, int N, int d, int block, int global_window, void* workspace,
+                    size_t ws_bytes, void* dq, void* dk, void* dv, void* stream, bool d_from_o) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_block(block, ASA_SAMPLES));
   const void* bf[] = {qp, kp, vp, o, dout, dq, dk, dv};
@@ -460,9 +459,29 @@ int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const vo
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
   e = asa::launch_bwd_tc(qp, kp, vp, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
                          d, global_window, workspace, dq, dk, dv, err_word, num_sms_current(),
-                         static_cast<cudaStream_t>(stream));
+                         static_cast<cudaStream_t>(stream), d_from_o ? o : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return ASA_OK;
+}
+
+int asa_sparse_attn_bwd(const void* qp, const void* kp, const void* vp, const void* o,
+                        const void* dout, const float* lse, const int32_t* row_ptr,
+                        const int32_t* col_idx, const int32_t* col_ptr_t,
+                        const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                        int global_window, void* workspace, size_t ws_bytes, void* dq, void* dk,
+                        void* dv, void* stream) {
+  return bwd_impl(qp, kp, vp, o, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B, H, N, d,
+                  block, global_window, workspace, ws_bytes, dq, dk, dv, stream, false);
+}
+
+int asa_sparse_attn_bwd_d_from_o(const void* qp, const void* kp, const void* vp, const void* o,
+                                 const void* dout, const float* lse, const int32_t* row_ptr,
+                                 const int32_t* col_idx, const int32_t* col_ptr_t,
+                                 const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                                 int global_window, void* workspace, size_t ws_bytes, void* dq,
+                                 void* dk, void* dv, void* stream) {
+  return bwd_impl(qp, kp, vp, o, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B, H, N, d,
+                  block, global_window, workspace, ws_bytes, dq, dk, dv, stream, true);
 }
 
 // ---------------------------------------------------------------- query pruning (BSA)

@@ -50,6 +50,8 @@
 // and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "softmax_math.cuh"
@@ -858,6 +860,36 @@ __global__ void __launch_bounds__(256)
 
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// D = rowsum(dO * O) from the stored bf16 O (the opt-in approximate D): one warp per
+// row, fp32 accumulation; rows past N keep the 0 of bwd_prep.
+template <int D>
+__global__ void __launch_bounds__(256)
+    d_from_o_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o,
+                    int64_t rows, int N, int Np, float* __restrict__ Dvec) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < rows; row += warps) {
+    const __nv_bfloat16* a = dout + row * D + lane * E;
+    const __nv_bfloat16* b = o + row * D + lane * E;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const uint32_t ua = *reinterpret_cast<const uint32_t*>(a + e);
+      const uint32_t ub = *reinterpret_cast<const uint32_t*>(b + e);
+      acc = fmaf(__uint_as_float(ua << 16), __uint_as_float(ub << 16), acc);
+      acc = fmaf(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      const int64_t bh = row / N;
+      Dvec[bh * Np + (row - bh * N)] = acc;
+    }
+  }
+}
+
 // Workspace pieces (256-byte aligned, in this order): lse2, D [BH][nbq*128] f32; Q16
 // [BH][Nq][d] f16, K16 [BH][N][d] f16; launch orders of query and key blocks
 // [BH*nbq], [BH*nbk] i32; with ASA_G (G global tokens): Kg, Vg [BH][G][d] bf16, Kg16
@@ -910,7 +942,7 @@ cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
                            const int32_t* col_ptr_t, const int32_t* row_idx_t,
                            const uint8_t* tquarters, const BwdWs& ws, int BH, int N, int Nq,
                            int G, int gw, void* dq, void* dk, void* dv, unsigned int* err_word,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool d_pass = true) {
   using L = BwdLayout<D>;
   const int nbq = (Nq + kBlock - 1) / kBlock;
   const int nbk = (N + kBlock - 1) / kBlock;
@@ -945,10 +977,12 @@ cudaError_t launch_kernels(const CUtensorMap* maps, const int32_t* row_ptr,
   if (regs_checked < 0) return cudaErrorInvalidConfiguration;
   const int grid_q = BH * nbq, grid_k = BH * nbk;
   // maps: Q16, dO, K16, V, Kg16, Vg (the last two stand in for K16, V without ASA_G)
-  bwd_row_kernel<D, true, kPruned><<<grid_q, kBwdThreads, L::kSmem, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, quarters, ws.ord_r,
-      N, Nq, nbq, Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, err_word, limit);
-  if ((e = cudaGetLastError())) return e;
+  if (d_pass) {  // otherwise D is already in ws.Dvec (rowsum(dO * O) from the stored O)
+    bwd_row_kernel<D, true, kPruned><<<grid_q, kBwdThreads, L::kSmem, stream>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], row_ptr, col_idx, quarters,
+        ws.ord_r, N, Nq, nbq, Np, G, gbias2, c2, scale, ws.lse2, ws.Dvec, nullptr, err_word, limit);
+    if ((e = cudaGetLastError())) return e;
+  }
   if (G > 0) {
     const int gtiles = BH * ((G + kBlock - 1) / kBlock);
     bwd_col_kernel<D, true><<<gtiles, kBwdThreads, L::kSmem, stream>>>(
@@ -1049,7 +1083,8 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk, void* dv,
-                          unsigned int* err_word, int num_sms, cudaStream_t stream) {
+                          unsigned int* err_word, int num_sms, cudaStream_t stream,
+                          const void* o_for_d) {
   const int nb = (N + kBlock - 1) / kBlock;
   const int Np = nb * kBlock;
   const int gw = global_window;
@@ -1066,12 +1101,25 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
   if (e == cudaSuccess && G > 0) e = global_tokens(kp, vp, ws, BH, N, d, gw, G, err_word, num_sms, stream);
   if (e == cudaSuccess) e = launch_lpt_order(row_ptr, BH, nb, nb, ws.ord_r, stream);
   if (e == cudaSuccess) e = launch_lpt_order(col_ptr_t, BH, nb, nb, ws.ord_c, stream);
+  if (e == cudaSuccess && o_for_d != nullptr) {
+    const int64_t rows = static_cast<int64_t>(BH) * N;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>((rows + 7) / 8, num_sms * 16));
+    const auto* a = static_cast<const __nv_bfloat16*>(dout);
+    const auto* b = static_cast<const __nv_bfloat16*>(o_for_d);
+    if (d == 128)
+      d_from_o_kernel<128><<<grid, 256, 0, stream>>>(a, b, rows, N, Np, ws.Dvec);
+    else
+      d_from_o_kernel<64><<<grid, 256, 0, stream>>>(a, b, rows, N, Np, ws.Dvec);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
+  const bool d_pass = o_for_d == nullptr;
   if (d == 128)
     return launch_kernels<128, false>(maps, row_ptr, col_idx, nullptr, col_ptr_t, row_idx_t,
-                                      nullptr, ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream);
+                                      nullptr, ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream,
+                                      d_pass);
   return launch_kernels<64, false>(maps, row_ptr, col_idx, nullptr, col_ptr_t, row_idx_t, nullptr,
-                                   ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream);
+                                   ws, BH, N, N, G, gw, dq, dk, dv, err_word, stream, d_pass);
 }
 
 // Backward with query pruning on the packed tiles of the pruned forward: the query

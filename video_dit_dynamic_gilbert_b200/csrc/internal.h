@@ -75,7 +75,8 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const float* lse, const int32_t* row_ptr, const int32_t* col_idx,
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk,
-                          void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream);
+                          void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream,
+                          const void* o_for_d = nullptr);
 
 // Gilbert gather from / scatter into per-rank token chunks: chunk s holds the rows
 // [B][tok.off[s+1] - tok.off[s]][H][d] of rank s's tokens, chunks back to back (the
