@@ -66,3 +66,19 @@ def test_autograd_equals_step_by_step():
     assert torch.equal(out.detach(), asa.asa_unpermute(op, wl.T, wl.Hg, wl.W))
     for t, gp in zip((q, k, v), grads):
         assert torch.equal(t.grad, asa.asa_unpermute(gp, wl.T, wl.Hg, wl.W))
+
+
+def test_autograd_d_from_o_equals_step_by_step():
+    wl = WORKLOADS["tiny"]
+    x = make_inputs(wl, with_dout=True)
+    q, k, v = (x[name].cuda().requires_grad_(True) for name in ("q", "k", "v"))
+    out = asa.asa_attention_trainable(q, k, v, wl.T, wl.Hg, wl.W, wl.tau, d_from_o=True)
+    out.backward(x["dout"].cuda())
+    qp, kp, vp = asa.asa_gilbert_permute3(q.detach(), k.detach(), v.detach(), wl.T, wl.Hg, wl.W)
+    m = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
+    op, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, m)
+    dop = asa.asa_gilbert_permute(x["dout"].cuda(), wl.T, wl.Hg, wl.W)
+    grads = asa.asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, m, d_from_o=True)
+    asa.asa_check_device_status()
+    for t, gp in zip((q, k, v), grads):
+        assert torch.equal(t.grad, asa.asa_unpermute(gp, wl.T, wl.Hg, wl.W))

@@ -537,7 +537,7 @@ class ASAAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
-                query_keep: float | None = None, query_window: int = 8):
+                query_keep: float | None = None, query_window: int = 8, d_from_o: bool = False):
         q, k, v = (t.contiguous() for t in (q, k, v))
         qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W)
         mask = asa_estimate_mask(qp, kp, tau, transposed=True)
@@ -551,6 +551,7 @@ class ASAAttention(torch.autograd.Function):
         ctx.save_for_backward(qp, kp, vp, op, lse)
         ctx.mask, ctx.grid, ctx.global_window, ctx.prune = mask, (T, Hg, W), global_window, prune
         ctx.tmask = tmask if prune is not None else None
+        ctx.d_from_o = d_from_o
         return asa_unpermute(op, T, Hg, W)
 
     @staticmethod
@@ -560,19 +561,21 @@ class ASAAttention(torch.autograd.Function):
         dop = asa_gilbert_permute(dout.to(torch.bfloat16).contiguous(), T, Hg, W)
         if ctx.prune is None:
             grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
-                                        global_window=ctx.global_window)
+                                        global_window=ctx.global_window, d_from_o=ctx.d_from_o)
         else:
             grads = asa_sparse_attn_bwd_pruned(ctx.prune, kp, vp, dop, lse, ctx.tmask,
                                                global_window=ctx.global_window)
         dq, dk, dv = (asa_unpermute(g, T, Hg, W) for g in grads)
-        return dq, dk, dv, None, None, None, None, None, None, None
+        return dq, dk, dv, None, None, None, None, None, None, None, None
 
 
 def asa_attention_trainable(q, k, v, T: int, Hg: int, W: int, tau: float,
                             global_window: int = 0, query_keep: float | None = None,
-                            query_window: int = 8):
+                            query_window: int = 8, d_from_o: bool = False):
     """Differentiable asa_attention: returns O [B, N, H, d] (raster); gradients flow to
     q, k and v through the kernels' backward under the forward's mask (and, with
-    query_keep, the forward's query pruning)."""
-    return ASAAttention.apply(q, k, v, T, Hg, W, tau, global_window, query_keep, query_window)
+    query_keep, the forward's query pruning).  d_from_o=True selects the faster,
+    less exact backward (D from the stored O; without query pruning)."""
+    return ASAAttention.apply(q, k, v, T, Hg, W, tau, global_window, query_keep, query_window,
+                              d_from_o)
 
