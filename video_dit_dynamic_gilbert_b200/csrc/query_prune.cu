@@ -11,6 +11,12 @@
 // tile runs over the union of its blocks' kept key blocks, and each key block of the
 // union carries a bit per 32-row TMEM lane quarter telling which rows may see it.
 // A pruned token then takes its centre's output row and LSE (token filling).
+//
+// Kernels: prune_kernel (selection and packing), pack_count/pack_fill (tile CSR with
+// quarter bits), fill_out_kernel (token filling of O and LSE); for the packed
+// backward, dout_compact_kernel (each kept row's summed output gradient and lse2 in
+// the compact layout), tile_dense/tile_transpose (the tile CSR per key block) and
+// dq_scatter_kernel (dQ back to every token, zero for pruned ones).
 #include "common.cuh"
 #include "internal.h"
 
