@@ -278,3 +278,17 @@ def test_seqpar_rejects(L):
                                   None) == asa.ASA_ERR_INVALID_ARG
     assert L.asa_seqpar_unpermute(FAKE, FAKE, 1, 0, 16, 16, 2, 64, offs(0, 1024), 1,
                                   None) == asa.ASA_ERR_INVALID_ARG
+
+
+def test_bwd_d_from_o_rejects(L):
+    # same contract as asa_sparse_attn_bwd: workspace, window and pointer checks first
+    args = [FAKE] * 10 + [1, 2, 1024, 64, 128, 0, None, 0] + [FAKE] * 3 + [None]
+    assert L.asa_sparse_attn_bwd_d_from_o(*args) == asa.ASA_ERR_WORKSPACE
+    args[15] = -1
+    assert L.asa_sparse_attn_bwd_d_from_o(*args) == asa.ASA_ERR_INVALID_ARG
+    args[15] = 0
+    args[3] = MIS     # o, the operand this variant reads
+    assert L.asa_sparse_attn_bwd_d_from_o(*args) == asa.ASA_ERR_INVALID_ARG
+    args[3] = FAKE
+    args[13] = 96     # d
+    assert L.asa_sparse_attn_bwd_d_from_o(*args) == asa.ASA_ERR_UNSUPPORTED
