@@ -35,3 +35,35 @@ def test_kept_tile_flops_small():
     L = [128, 128, 44]
     want = 4 * 64 * (L[0] * L[0] + L[0] * L[2] + L[2] * L[1] + L[2] * L[2])
     assert (flops, nnz, tiles) == (want, 4, 9)
+
+
+def _csr(mask):
+    rows = mask.reshape(-1, mask.shape[-1])
+    rp = np.concatenate([[0], np.cumsum(rows.sum(1))]).astype(np.int64)
+    ci = np.concatenate([np.nonzero(r)[0] for r in rows]).astype(np.int64)
+    return rp, ci
+
+
+def test_pruned_flops_against_kept_tile_flops():
+    B, H, N, d = 1, 2, 300, 64            # blocks of 128, 128, 44
+    g = np.random.default_rng(3)
+    mask = g.random((B, H, 3, 3)) < 0.6
+    mask[..., np.arange(3), np.arange(3)] = True
+    rp, ci = _csr(mask)
+    full, _, _ = bench._kept_tile_flops(rp, ci, B, H, N, d)
+    # every query kept: the kept-tile count
+    src_all = np.tile(np.arange(N), (B, H, 1))
+    f_all, kept_all = bench._pruned_flops(rp, ci, src_all, B, H, N, d)
+    assert f_all == full and kept_all == B * H * N
+    # every other token points at its left neighbour: half of each even block kept
+    src_half = src_all.copy()
+    src_half[..., 1::2] -= 1
+    f_half, kept_half = bench._pruned_flops(rp, ci, src_half, B, H, N, d)
+    assert kept_half == B * H * N // 2
+    L = np.array([128, 128, 44])
+    K = L // 2
+    expect = 0
+    for h in range(H):
+        for I in range(3):
+            expect += 4 * d * K[I] * L[np.nonzero(mask[0, h, I])[0]].sum()
+    assert f_half == expect
