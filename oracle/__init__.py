@@ -23,6 +23,16 @@ Parity status per function (how each is pinned is in tests/test_oracle_*.py):
                      in-block permutation invariance.
   build_mask         pinned: brute-force minimality over all subsets (nb=8),
                      tau->0 keeps the argmax, tau=1 keeps all, monotone in tau.
+  marginal_rows      pinned: hand-built rows whose cumulative share lands 5e-5 and
+                     2e-4 from tau at the cut and one block before it, exact and
+                     near ties at the cut, tau = 1 (tests/golden/marginal_rows.json).
+  marginal_rows_stat pinned: hand-built rows with a share on the threshold, 4e-4
+                     from it, a fallback row with a tied and an untied maximum,
+                     k >= n (same fixture).
+  legal_mask_rows    pinned: hand-built rows and kept sets (a prefix one block short
+                     or long within and beyond 1e-4 of tau, a swap of near-equal and
+                     of distinct shares, a size off by more than one, tau = 1); the
+                     exact cut is legal on random rows (same fixture).
   asa_forward        pinned: tau=1 equals dense attention (torch SDPA fp64);
                      any mask equals SDPA with the token-expanded block mask.
   asa_g_forward      pinned: SDPA fp64 over Concat(K, MeanPool_n K) with the
@@ -56,6 +66,7 @@ from .asa_ref import (  # noqa: F401
     mask_to_csr,
     mask_to_csr_transposed,
     marginal_rows,
+    legal_mask_rows,
     global_tokens,
     round_to_bf16,
     asa_forward,

@@ -12,7 +12,7 @@ Video Generation" (arXiv 2508.10774), section "Adaptive Block-Sparse Attention":
     and ASA_G)
   * "Implementation details": b = 128, k = 16.
 
-Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
+Readings taken where the pages are silent:
   * blocks are consecutive runs of b permuted tokens; the last block is ragged,
     nothing is padded;
   * the k "representative tokens" of a block of L tokens are the evenly strided
@@ -245,6 +245,48 @@ def marginal_rows(pimp: np.ndarray, tau: float, eps: float = 1e-4,
                     m |= abs(share[order[c - 1]] - share[order[c]]) < tie_eps
                 marg[bb, h, I] = m
     return marg
+
+
+def legal_mask_rows(pimp: np.ndarray, mask: np.ndarray, tau: float, eps: float = 1e-4,
+                    tie_rel: float = 5e-4) -> np.ndarray:
+    """Rows of a block mask [B, H, nb, nb] that are a legal threshold cut of ``pimp``
+    under a small perturbation of its values ("Step 2.1": the fewest blocks, taken in
+    descending order, whose cumulative share reaches tau).
+
+    A row's kept set S is legal when, with the row's exact shares R:
+      * tau >= 1: S is every block;
+      * |S| differs from the exact cut c* by at most one;
+      * S is a leading set of the descending order up to near-ties: the smallest
+        share in S is at least (1 - tie_rel) times the largest share left out;
+      * S reaches tau within eps: sum_S R >= tau - eps;
+      * S is minimal within eps: without its smallest share it stays below
+        tau + eps.
+    The exact cut of build_mask satisfies all five.  A set evaluated from shares
+    that carry a relative error well below tie_rel (an fp32 estimate) can differ
+    from it only at a row whose cumulative share at the cut is within eps of tau,
+    or by the order of near-equal shares, and still passes.  Returns [B, H, nb] bool.
+    """
+    B, H, nb, _ = pimp.shape
+    ok = np.zeros((B, H, nb), dtype=bool)
+    for bb in range(B):
+        for h in range(H):
+            for I in range(nb):
+                S = np.asarray(mask[bb, h, I], dtype=bool)
+                if tau >= 1.0:
+                    ok[bb, h, I] = bool(S.all())
+                    continue
+                if not S.any():
+                    continue
+                share, order = _row_order(pimp[bb, h, I])
+                c = _row_cut(share, order, tau)
+                if abs(int(S.sum()) - c) > 1:
+                    continue
+                smin = share[S].min()
+                if (~S).any() and smin < (1.0 - tie_rel) * share[~S].max():
+                    continue
+                cum = share[S].sum()
+                ok[bb, h, I] = cum >= tau - eps and cum - smin < tau + eps
+    return ok
 
 
 def mask_to_csr(mask: np.ndarray):

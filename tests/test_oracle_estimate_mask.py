@@ -226,3 +226,66 @@ def test_stat_mask_quantile_matches_table_values():
     want = s >= s.mean() + s.std() * 0.674490
     assert 0 < want.sum() < n
     assert m[0, 0, 0].tolist() == want.tolist()
+
+
+# ---------------------------------------------------------------- marginal / legal rows
+
+def _fixture():
+    with open(os.path.join(GOLDEN, "marginal_rows.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _fixture()["marginal"], ids=lambda c: c["why"][:40])
+def test_marginal_rows_hand_built(case):
+    row = np.asarray(case["p_imp"], dtype=np.float64)
+    got = oracle.marginal_rows(row[None, None, None, :], case["tau"])
+    assert bool(got[0, 0, 0]) is case["marginal"], case["why"]
+
+
+@pytest.mark.parametrize("case", _fixture()["marginal_stat"], ids=lambda c: c["why"][:40])
+def test_marginal_rows_stat_hand_built(case):
+    row = np.asarray(case["p_imp"], dtype=np.float64)
+    got = oracle.marginal_rows_stat(row[None, None, None, :], case["k"])
+    assert bool(got[0, 0, 0]) is case["marginal"], case["why"]
+
+
+def test_marginal_rows_stat_fallback_row_keeps_lowest_maximum():
+    # the tied fallback row of the fixture keeps J0, the lowest of the equal maxima
+    m = oracle.build_mask_stat(np.asarray([0.3, 0.3, 0.3, 0.1])[None, None, None, :], 1)
+    assert np.nonzero(m[0, 0, 0])[0].tolist() == [0]
+
+
+@pytest.mark.parametrize("case", _fixture()["legal"], ids=lambda c: c["why"][:40])
+def test_legal_mask_rows_hand_built(case):
+    row = np.asarray(case["p_imp"], dtype=np.float64)
+    S = np.zeros(len(row), dtype=bool)
+    S[case["kept"]] = True
+    got = oracle.legal_mask_rows(row[None, None, None, :], S[None, None, None, :], case["tau"])
+    assert bool(got[0, 0, 0]) is case["legal"], case["why"]
+
+
+def test_legal_mask_rows_accepts_exact_cut_and_rejects_perturbed_sets():
+    """The exact cut is legal on every row; dropping its largest block, or adding the
+    largest dropped block when that block is far from a tie and the cut is far from tau,
+    is not."""
+    g = np.random.default_rng(21)
+    pimp = g.random((1, 2, 24, 24)) ** 4 + 1e-4
+    for tau in (0.5, 0.8, 0.95):
+        m = oracle.build_mask(pimp, tau)
+        assert oracle.legal_mask_rows(pimp, m, tau).all()
+        marg = oracle.marginal_rows(pimp, tau)
+        for h in range(2):
+            for I in range(24):
+                share = pimp[0, h, I] / pimp[0, h, I].sum()
+                bad = m[0, h, I].copy()
+                bad[int(np.argmax(share))] = False
+                if bad.any():
+                    assert not oracle.legal_mask_rows(pimp[:, h:h + 1, I:I + 1],
+                                                      bad[None, None, None], tau)[0, 0, 0]
+                if not marg[0, h, I] and (~m[0, h, I]).any():
+                    extra = m[0, h, I].copy()
+                    extra[int(np.argmax(np.where(m[0, h, I], -1.0, share)))] = True
+                    cum = share[m[0, h, I]].sum()
+                    if cum - tau > 1e-3:
+                        assert not oracle.legal_mask_rows(pimp[:, h:h + 1, I:I + 1],
+                                                          extra[None, None, None], tau)[0, 0, 0]
