@@ -30,7 +30,23 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "wan2.1-1.3b"
 METRIC = "ASA ms/call & effective TFLOP/s at 32760 tok, H=12, d=128, τ=0.95"
-KERNELS_PER_STEP = 11  # permute3, est_gather, est_tc, est_combine, est_pool, mask_rows, scan, fill, lpt_order, fwd, unpermute
+
+
+def count_launches(torch, step):
+    """Kernels of this library (namespace asa) that one step launches, counted by CUPTI
+    through torch.profiler over one untimed step: (count, sorted distinct names), or
+    (None, reason) when the profiler is unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events()
+                 if "asa::" in e.name and str(e.device_type).endswith("CUDA")]
+        return len(names), sorted(set(n.split("(")[0][-60:] for n in names))
+    except Exception as exc:  # noqa: BLE001 - report, do not fail the bench
+        return None, f"profiler unavailable: {type(exc).__name__}"
 
 
 def _peaks():
@@ -137,9 +153,9 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": n, "samples_under_load": len(sm)}
 
 
-def oracle_setup(wl, x, h=0):
+def oracle_setup(wl, x, h=0, with_pimp=False):
     """The oracle's permuted Q, K, V of head h and its estimate + mask, with the time
-    the estimate + mask took."""
+    the estimate + mask took (and the oracle's P_imp when asked)."""
     import oracle
     perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
     t0 = time.perf_counter()
@@ -147,7 +163,27 @@ def oracle_setup(wl, x, h=0):
                   for n in ("q", "k", "v"))
     pimp = oracle.estimate_pimp(qp, kp)
     mask = oracle.build_mask(pimp, wl.tau)
-    return qp, kp, vp, mask, time.perf_counter() - t0
+    out = (qp, kp, vp, mask, time.perf_counter() - t0)
+    return out + (pimp,) if with_pimp else out
+
+
+def mask_rows_vs_oracle(wl, pimp, mask, row_ptr, col_idx, h=0):
+    """Rows of head h of the timed call's mask against the oracle's: how many differ,
+    how many the oracle marks marginal, and how many differing rows are not a legal cut
+    of the oracle's P_imp (a leading set within near-ties, one block from the exact cut
+    at most, reaching tau within 1e-4 and minimal within 1e-4)."""
+    import oracle
+    nb = mask.shape[-1]
+    rp = row_ptr.astype(np.int64)
+    gm = np.zeros((1, 1, nb, nb), dtype=bool)
+    for I in range(nb):
+        gm[0, 0, I, col_idx[rp[h * nb + I]:rp[h * nb + I + 1]]] = True
+    differ = (gm != mask).any(-1)
+    marg = oracle.marginal_rows(pimp, wl.tau)
+    legal = oracle.legal_mask_rows(pimp, gm, wl.tau)
+    return {"head": h, "differ": int(differ.sum()), "marginal": int(marg.sum()),
+            "differ_not_marginal": int((differ & ~marg).sum()), "not_legal": int((~legal).sum()),
+            "of": int(nb)}
 
 
 def cpu_oracle_sample(wl, x, budget_s=15.0, setup=None, seed=0):
@@ -285,7 +321,8 @@ class _Timer:
 
 
 def _report_config(asa, torch, wl, timer, dev, peaks):
-    """Every stage of one workload, timed separately (SURVEY-style split)."""
+    """Every stage of one workload, timed separately (permute, estimate, mask,
+    attention, pool, backward, unpermute)."""
     from inputs import make_inputs
     x = make_inputs(wl, with_dout=wl.backward)
     q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
@@ -643,8 +680,12 @@ def main():
                      "peak_kind": f"{peak_kind} bf16 burst",
                      "frac_of_sustained": achieved / sustained},
         "clocks": clk,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
     }
+    per_step, names = count_launches(torch, step)
+    result["gpu_launches"] = per_step * args.steps if per_step is not None else None
+    result["gpu_launches_how"] = (f"{per_step} kernels of this library per step, counted by "
+                                  f"CUPTI (torch.profiler) over one untimed step, x steps"
+                                  if per_step is not None else names)
 
     # ---- end to end through the public host-buffer call (asa_attention_host): pinned
     # raster Q, K, V in, raster O out, the library's copies pipelined against its
@@ -707,7 +748,10 @@ def main():
         result["extras"]["host_sequential_ms"] = statistics.median(seq)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_oracle_sample(wl, x)
+        *setup, pimp0 = oracle_setup(wl, x, with_pimp=True)
+        result["cpu_baseline"] = cpu_oracle_sample(wl, x, setup=tuple(setup))
+        result["mask_rows"] = mask_rows_vs_oracle(wl, pimp0, setup[3], mask.row_ptr.cpu().numpy(),
+                                                  mask.col_idx.cpu().numpy())
     if rank == 0:
         print(json.dumps(result))
     if world > 1:

@@ -26,3 +26,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Mask rows that differ from the oracle's (each one checked to be a legal cut)."""
+    import mask_report
+    if not mask_report.RECORDS:
+        return
+    tr = terminalreporter
+    tr.section("mask rows against the oracle (differing rows are legal cuts)")
+    tot = [0, 0, 0]
+    for what, differ, marginal, rows in mask_report.RECORDS:
+        tr.write_line(f"{what}: {differ} differ, {marginal} marginal, of {rows} rows")
+        tot = [tot[0] + differ, tot[1] + marginal, tot[2] + rows]
+    tr.write_line(f"total: {tot[0]} differ, {tot[1]} marginal, of {tot[2]} rows")

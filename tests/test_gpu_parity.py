@@ -2,20 +2,24 @@
 on the same seeded inputs, at sizes the oracle finishes in seconds that still span
 several blocks and a ragged tail, plus the degenerate cases.
 
-Bars: permutations and CSR masks bit-exact (mask rows may differ only where the
-oracle marks the row marginal); outputs and gradients max-abs <= 2e-2 and rel-L2 <=
-5e-3 against the oracle using the oracle's mask; LSE within 1e-3."""
+Bars: permutations and CSR masks bit-exact.  From the oracle's own P_imp (rounded to
+fp32) the mask kernel must reproduce the oracle's cut on every row; through the
+library's fp32 estimate a row may differ only where the oracle marks it marginal, and
+then it must still be a legal cut of the oracle's P_imp.  Outputs and gradients:
+max-abs <= 2e-2 and rel-L2 <= 5e-3 against the oracle using the oracle's mask; LSE
+within 1e-3."""
 import math
 
 import numpy as np
 import pytest
 import torch
 
+import mask_report
 import oracle
 from inputs import WORKLOADS, make_inputs
 from video_dit_dynamic_gilbert_b200 import asa
-from gpu_util import (LSE_ABS, check_close, check_transposed, compare_masks, f64, mask_from_csr,
-                      upload_mask)
+from gpu_util import (LSE_ABS, check_close, check_close_ulp, check_transposed, compare_masks,
+                      f64, mask_from_csr, upload_mask)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,7 +85,7 @@ def test_mask_bit_exact(name, tau):
     kp = torch.from_numpy(ref["k"]).to(torch.bfloat16).cuda()
     bm = asa.asa_estimate_mask(qp, kp, t, transposed=True)
     gm = mask_from_csr(bm)
-    compare_masks(gm, mask, marg)
+    compare_masks(gm, mask, marg, pimp, t, what=f"{name} tau={t}")
     assert int(bm.nnz.item()) == int(gm.sum())
     check_transposed(bm, gm)
     if t >= 1.0:
@@ -90,6 +94,60 @@ def test_mask_bit_exact(name, tau):
     p = asa.asa_estimate(qp, kp)
     bm2 = asa.asa_build_mask(p, wl.N, t)
     assert np.array_equal(mask_from_csr(bm2), gm)
+
+
+def kernel_only_mask(pimp, N, tau, what):
+    """The mask kernel alone on the oracle's P_imp rounded to fp32, against the oracle's
+    cut of the same fp32 values at the fp32 value of tau (the kernel's tau argument is a
+    float).  Rows must be identical except where the fp64 cumulative share at the cut, or
+    one block before it, lies within 1e-12 of tau: there the order of the fp64
+    additions decides (the kernel sums raw values against tau * total, the oracle sums
+    shares).  Exact ties are decided alike (lower J first) and are not excused."""
+    t32 = float(np.float32(tau))
+    p32 = np.ascontiguousarray(pimp, dtype=np.float32)
+    p64 = p32.astype(np.float64)
+    bm = asa.asa_build_mask(torch.from_numpy(p32).cuda(), N, tau, transposed=True)
+    asa.asa_check_device_status()
+    got = mask_from_csr(bm)
+    want = oracle.build_mask(p64, t32)
+    tight = oracle.marginal_rows(p64, t32, eps=1e-12, tie_eps=0.0)
+    differ = (got != want).any(-1)
+    assert not (differ & ~tight).any(), (f"{what}: {int((differ & ~tight).sum())} rows differ, "
+                                        f"e.g. {np.argwhere(differ & ~tight)[:5]}")
+    assert int(bm.nnz.item()) == int(got.sum())
+    check_transposed(bm, got)
+    mask_report.record(f"kernel only, {what}", differ.sum(), tight.sum(), differ.size)
+    return got
+
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("tau", [None, 0.5, 0.8, 0.99, 1.0, 1e-6])
+def test_mask_kernel_bit_exact_from_oracle_pimp(name, tau):
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    t = wl.tau if tau is None else tau
+    got = kernel_only_mask(pimp, wl.N, t, f"{name} tau={t}")
+    if t >= 1.0:
+        assert got.all()
+
+
+def test_mask_kernel_ties_and_ragged_rows():
+    """Rows with exact ties at the cut (equal fp32 values: the lower J is kept first), a
+    row whose values are all equal, a row of one dominant block, and nb = 3 (a grid
+    smaller than one warp's stride)."""
+    nb = 40
+    g = np.random.default_rng(5)
+    p = (g.random((1, 2, nb, nb)) ** 3).astype(np.float32)
+    p[0, 0, 0] = 1.0                                   # all equal: any tau < 1 keeps a prefix in J
+    p[0, 0, 1] = 1e-6
+    p[0, 0, 1, 7] = 1.0                                # one dominant block
+    p[0, 0, 2, ::2] = 0.25                             # ties straddling the cut
+    p[0, 1, 3] = np.repeat(np.arange(nb // 4, dtype=np.float32), 4)[::-1] + 1
+    for tau in (0.3, 0.5, 0.9, 0.97):
+        kernel_only_mask(p, 128 * nb, tau, f"ties tau={tau}")
+    small = (g.random((2, 3, 3, 3)) + 0.1).astype(np.float32)
+    small[0, 0, 0] = 1.0
+    for tau in (0.2, 0.6, 0.95):
+        kernel_only_mask(small, 3 * 128 - 5, tau, f"nb=3 tau={tau}")
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -206,6 +264,10 @@ def test_backward_unkept_key_blocks(name):
         check_close(f64(g), e, what=what)
     assert (f64(got[1])[:, :, 128 * (nb - 1):] == 0).all()
     assert (f64(got[2])[:, :, 128 * (nb - 1):] == 0).all()
+    # unscaled dO: the fixed absolute bar widened by one bf16 ulp of the reference
+    _, got1, exp1 = _backward_pair(name, mask, dout_scale=1.0)
+    for g, e, what in zip(got1, exp1, ("dQ", "dK", "dV")):
+        check_close_ulp(f64(g), e, what=f"{what} unscaled")
 
 
 @pytest.mark.parametrize("name", ["one-ragged-block", "d128-ragged"])
@@ -251,6 +313,14 @@ def test_asa_g_backward_with_oracle_mask(name, n):
     check_close(dq, rq, what="ASA_G dQ")
     check_close(dk, rk, what="ASA_G dK")
     check_close(dv, rv, what="ASA_G dV")
+    if sc != 1.0:
+        # unscaled dO: the fixed absolute bar widened by one bf16 ulp of the reference
+        dop1 = torch.from_numpy(ref["dout"]).to(torch.bfloat16).cuda()
+        got1 = [f64(t) for t in asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop1, lse, bm,
+                                                        global_window=n)]
+        asa.asa_check_device_status()
+        for g, e, what in zip(got1, (rq, rk, rv), ("dQ", "dK", "dV")):
+            check_close_ulp(g, e / sc, what=f"ASA_G {what} unscaled")
 
 
 def test_backward_deterministic():
@@ -285,15 +355,14 @@ def test_end_to_end_call(name):
     wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
     out, lse, bm = asa.asa_attention(dev["q"], dev["k"], dev["v"], wl.T, wl.Hg, wl.W, wl.tau)
     gm = mask_from_csr(bm)
-    compare_masks(gm, mask, marg)
-    O_ref, _ = oracle.asa_forward(ref["q"], ref["k"], ref["v"], mask)
-    # query blocks whose (marginal) mask row differs are left out of the comparison
-    agree = ~(gm != mask).any(axis=-1)                       # [B, H, nb]
+    compare_masks(gm, mask, marg, pimp, wl.tau, what=f"{name} end to end")
+    # every row against the oracle's forward under the library's mask: equal to the
+    # oracle's mask except on marginal rows, where it was just checked to be a legal cut
+    O_ref, _ = oracle.asa_forward(ref["q"], ref["k"], ref["v"], gm)
     got = f64(out)                                           # raster [B, N, H, d]
     for bb in range(wl.B):
         for h in range(wl.H):
-            rows = np.nonzero(np.repeat(agree[bb, h], 128)[:wl.N])[0]
-            check_close(got[bb, perm[rows], h], O_ref[bb, h, rows], what="O end-to-end")
+            check_close(got[bb, perm, h], O_ref[bb, h], what="O end-to-end")
     asa.asa_check_device_status()
 
 
