@@ -130,14 +130,16 @@ int asa_build_mask(const float* p_imp, int B, int H, int N, float tau, void* wor
  * must not risk the synchronisation cudaMalloc may cause).  The paper has no
  * counterpart: this is a library convenience.  Same arguments, layouts and result
  * as asa_estimate minus the workspace.
- *   - Scratch: one file-scope device array of ASA_NOALLOC_SCRATCH_BYTES, reserved on
- *     every device that loads the library and held until the process exits.  Shapes
- *     needing more (about 6.2 MB per head at N = 32,760 and d = 128, i.e. at most 5
- *     heads per call at that shape) are rejected with ASA_ERR_WORKSPACE before
+ *   - Scratch: one file-scope device array of ASA_NOALLOC_SCRATCH_BYTES.  Under CUDA's
+ *     lazy module loading (the default) it is reserved on a device when the library's
+ *     module is first loaded there, which the first call on that device does, and it
+ *     is held until the process exits.  That first call may therefore reserve the
+ *     32 MiB and synchronise: make it during set-up, before any stream capture.
+ *     Shapes needing more (about 6.2 MB per head at N = 32,760 and d = 128, i.e. at
+ *     most 5 heads per call at that shape) are rejected with ASA_ERR_WORKSPACE before
  *     anything is launched.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address in the current context (the
+ *     address is not cached, so it stays valid across a context re-creation).
  *   - Every call shares the array and overwrites what it reads (nothing in it needs to
  *     start at zero).  Calls whose kernels overlap on the GPU (different streams, or
  *     several host threads) race on the array: serialise them.

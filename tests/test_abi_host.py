@@ -292,3 +292,12 @@ def test_bwd_d_from_o_rejects(L):
     args[3] = FAKE
     args[13] = 96     # d
     assert L.asa_sparse_attn_bwd_d_from_o(*args) == asa.ASA_ERR_UNSUPPORTED
+
+
+def test_trainable_op_rejects_d_from_o_with_query_pruning():
+    """The query-pruned backward always takes the exact D, so asking for both is an
+    error, raised before any device work."""
+    import torch
+    x = torch.zeros((1, 8, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        asa.asa_attention_trainable(x, x, x, 1, 2, 4, 0.9, query_keep=0.5, d_from_o=True)

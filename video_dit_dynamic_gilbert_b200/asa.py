@@ -538,6 +538,9 @@ class ASAAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
                 query_keep: float | None = None, query_window: int = 8, d_from_o: bool = False):
+        if d_from_o and query_keep is not None:
+            raise ValueError("d_from_o applies to the unpruned backward only; the query-pruned "
+                             "backward always takes the exact D")
         q, k, v = (t.contiguous() for t in (q, k, v))
         qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W)
         mask = asa_estimate_mask(qp, kp, tau, transposed=True)

@@ -1,6 +1,4 @@
 // Allocation-free variant of asa_estimate (the estimator itself is in estimate_tc.cu).
-#include <mutex>
-
 #include "../../include/asa.h"
 #include "common.cuh"
 #include "internal.h"
@@ -15,34 +13,26 @@
 // cause.  For them the estimator's scratch (the compact sample rows, per sample row the
 // max logit of every key block and the row's log2-sum-exp) lives in one file-scope
 // device array of fixed
-// size, reserved when the library is loaded on a device and held until the process
-// exits.  The caller still passes the inputs and the P_imp output.
+// size.  With CUDA's lazy module loading (the default) the array is reserved on a
+// device when this file's module is first loaded there, i.e. at the first call on that
+// device, and held until the process exits; that first call may synchronise, so make
+// it during set-up.  The caller still passes the inputs and the P_imp output.
 namespace {
 
 constexpr size_t kNoallocScratchFloats = ASA_NOALLOC_SCRATCH_BYTES / sizeof(float);
 static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
 
-std::mutex g_noalloc_mu;
-float* g_noalloc_addr[64] = {nullptr};
-
-// Device address of the scratch array on the current device, looked up once per
-// device (the host-side name of the array is not a device address).
+// Device address of the scratch array in the current context, looked up on every call
+// (the host-side name of the array is not a device address).  Nothing is cached: a
+// cached address would go stale when the context is torn down and re-created
+// (cudaDeviceReset), and the lookup itself allocates nothing.
 int noalloc_scratch(float** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess)
-    return asa::record_error(ASA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= 64) return asa::record_error(ASA_ERR_UNSUPPORTED, "device %d >= 64", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return asa::record_error(ASA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s",
-                               cudaGetErrorString(e));
-    g_noalloc_addr[dev] = static_cast<float*>(p);
-  }
-  *out = g_noalloc_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return asa::record_error(ASA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s",
+                             cudaGetErrorString(e));
+  *out = static_cast<float*>(p);
   return ASA_OK;
 }
 
