@@ -2,7 +2,7 @@
 
 The pages measure on real Wan2.1 / CogVideoX activations (JourneyDB prompts,
 VBench suites) that are not available; these seeded fields stand in for them.
-Recipe (also in DESIGN.md, "Inputs"):
+Recipe:
 
   F[t, y, x] = sum_m a_m cos(2 pi (f_t t / T + f_y y / H + f_x x / W) + phi_m)
       a_m ~ N(0, 1/M_m) in R^d, integer frequencies f uniform in [0, 3],

@@ -5,7 +5,7 @@ Locality-preserving token rearrangement": the flattened (T, H, W) video tokens a
 reordered along a Gilbert space-filling curve before they are cut into blocks, so
 that each block holds spatially contiguous tokens.  The pages name the curve but
 do not define it, so this module restates a generalised Hilbert construction of
-our own (the rules are written out in DESIGN.md, "Gilbert order"):
+our own:
 
 * A box is an origin ``o``, a signed major direction ``a`` of length ``P`` and two
   signed minor directions ``b`` (length ``Q``) and ``c`` (length ``R``).  The path

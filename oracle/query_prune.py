@@ -9,7 +9,7 @@ Layered on ASA's blocks ("Video-BLADE: Block-Sparse Attention Meets Step
 Distillation for Efficient Video Generation", "Preprocessing": runs of b = 128
 Gilbert-ordered tokens).
 
-Readings taken where the pages are silent (listed in DESIGN.md, "Readings"):
+Readings taken where the pages are silent:
   * a query block is a block of b permuted tokens; its windows are runs of w
     consecutive permuted tokens from the block start (the last one ragged);
     the centre of a window of length l starting at s is the token at s + l // 2;

@@ -2,8 +2,7 @@
 //
 // Video-BLADE, "Preprocessing: Locality-preserving token rearrangement": tokens are
 // reordered along a Gilbert space-filling curve before blocking.  The pages do not
-// define the curve; this is our own construction (rules in DESIGN.md, "Gilbert
-// order"), walked with an explicit stack:
+// define the curve; this is our own construction, walked with an explicit stack:
 //   box = origin o, major direction a (length P), minor directions b (Q), c (R);
 //   the walk enters at o and leaves at o + (P-1) a.
 //   Q == R == 1          -> straight run along a;
