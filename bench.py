@@ -791,6 +791,16 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
                                                         d_from_o=True), reps=5)
     flops, _, _ = _kept_tile_flops(tmask.row_ptr.cpu().numpy(), tmask.col_idx.cpu().numpy(),
                                    B, H, N, d)
+    # the training pair: forward with the fp32 output, backward taking D from it
+    tws = asa.fwd_train_workspace(B, H, N, d, 0, dev)
+    t_o, t_lse = torch.empty_like(qp), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    t_o32 = torch.empty(qp.shape, dtype=torch.float32, device=dev)
+    fwd_train_ms = timeit(lambda: asa.asa_sparse_attn_fwd_train(qp, kp, vp, tmask, workspace=tws,
+                                                                out=t_o, lse=t_lse, out32=t_o32))
+    bws = asa.bwd_workspace(B, H, N, d, dev)
+    t_grads = tuple(torch.empty_like(qp) for _ in range(3))
+    bwd_train_ms = timeit(lambda: asa.asa_sparse_attn_bwd_train(qp, kp, vp, t_o32, dout, t_lse, tmask,
+                                                                workspace=bws, outs=t_grads), reps=5)
     # ASA_G backward (n = 64) on the same mask
     og, lg = asa.asa_sparse_attn_fwd(qp, kp, vp, tmask, global_window=64)
     bwd_g_ms = timeit(lambda: asa.asa_sparse_attn_bwd(qp, kp, vp, og, dout, lg, tmask,
@@ -832,6 +842,8 @@ def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):
         "asa_g_fwd_tflops": (flops + 4 * d * N * G * B * H) / g_ms / 1e9,
         "bwd_ms": bwd_ms, "bwd_tflops": 2.5 * flops / bwd_ms / 1e9,
         "bwd_d_from_o_ms": bwd_dfo_ms, "bwd_d_from_o_tflops": 2.5 * flops / bwd_dfo_ms / 1e9,
+        "fwd_train_ms": fwd_train_ms, "fwd_train_tflops": flops / fwd_train_ms / 1e9,
+        "bwd_train_ms": bwd_train_ms, "bwd_train_tflops": 2.5 * flops / bwd_train_ms / 1e9,
         "asa_g_bwd_ms_n64": bwd_g_ms,
         "asa_g_bwd_tflops": 2.5 * (flops + 4 * d * N * G * B * H) / bwd_g_ms / 1e9,
     }

@@ -199,6 +199,29 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
                         void* stream);
 
 /*
+ * Workspace bytes of asa_sparse_attn_fwd_train (0 for invalid sizes): those of
+ * asa_sparse_attn_fwd plus an fp16 copy of V (B*H*N*d * 2 bytes) and, with
+ * global_window = n > 0, an fp16 copy of the G global V tokens (B*H*G*d * 2 bytes).
+ */
+size_t asa_fwd_train_workspace_size(int B, int H, int N, int d, int global_window);
+
+/*
+ * The forward of asa_sparse_attn_fwd (same computation, arguments, layouts and errors)
+ * for training: it also writes o32, the output in fp32 before its bf16 rounding, from
+ * which asa_sparse_attn_bwd_train takes D = rowsum(dO * O) ("Step 2.1": the mask of
+ * the forward restricts the backward too; D is the row term of the softmax gradient).
+ * For that D to be accurate, the P V product takes P in fp16 (11 significant bits, the
+ * inference forward's bf16 has 8) against an fp16 copy of V made in the workspace; V
+ * magnitudes must therefore stay at or below 65504 (a larger value is reported by the
+ * next asa_check_device_status as ASA_ERR_INVALID_ARG).  o: device bf16 [B, H, N, d];
+ * lse: device fp32 [B, H, N]; o32: device fp32 [B, H, N, d], 16-byte aligned.
+ */
+int asa_sparse_attn_fwd_train(const void* qp, const void* kp, const void* vp,
+                              const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N,
+                              int d, int block, int global_window, void* workspace,
+                              size_t ws_bytes, void* o, float* lse, float* o32, void* stream);
+
+/*
  * Workspace bytes of asa_sparse_attn_bwd (0 for invalid sizes): per-row lse*log2(e)
  * and D (fp32, rows padded to whole blocks), fp16 copies of Q and K
  * (2 * B*H*N*d * 2 bytes), and the launch orders of query and key blocks; with
@@ -250,6 +273,23 @@ int asa_sparse_attn_bwd_d_from_o(const void* qp, const void* kp, const void* vp,
                                  const int32_t* row_idx_t, int B, int H, int N, int d, int block,
                                  int global_window, void* workspace, size_t ws_bytes, void* dq,
                                  void* dk, void* dv, void* stream);
+
+/*
+ * asa_sparse_attn_bwd for a forward run by asa_sparse_attn_fwd_train: D is taken as
+ * rowsum(dO * O) from that forward's fp32 output o32 (device fp32 [B, H, N, d]) in one
+ * pass over dO and o32, instead of the exact pass over the kept tiles (two GEMMs per
+ * kept tile).  The gradients meet the same tolerances as asa_sparse_attn_bwd's (the
+ * fp16 P of that forward leaves O within ~2^-12 relative of its exact value); dV does
+ * not depend on D and is bit-identical to asa_sparse_attn_bwd's.  Same workspace
+ * (asa_bwd_workspace_size), arguments and errors as asa_sparse_attn_bwd, with o32 in
+ * place of o; lse must come from the same training forward.  Deterministic.
+ */
+int asa_sparse_attn_bwd_train(const void* qp, const void* kp, const void* vp, const float* o32,
+                              const void* dout, const float* lse, const int32_t* row_ptr,
+                              const int32_t* col_idx, const int32_t* col_ptr_t,
+                              const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                              int global_window, void* workspace, size_t ws_bytes, void* dq,
+                              void* dk, void* dv, void* stream);
 
 /* ------------------------------------------------------------------------------
  * Query pruning with token filling ("Bidirectional Sparse Attention for Faster

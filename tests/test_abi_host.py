@@ -301,3 +301,26 @@ def test_trainable_op_rejects_d_from_o_with_query_pruning():
     x = torch.zeros((1, 8, 2, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         asa.asa_attention_trainable(x, x, x, 1, 2, 4, 0.9, query_keep=0.5, d_from_o=True)
+
+
+def test_training_pair_rejects(L):
+    # forward: workspace first, then the fp32 output's alignment, then d
+    args = [FAKE] * 5 + [1, 2, 1024, 64, 128, 0, None, 0, FAKE, FAKE, FAKE, None]
+    assert L.asa_sparse_attn_fwd_train(*args) == asa.ASA_ERR_WORKSPACE
+    need = L.asa_fwd_train_workspace_size(1, 2, 1024, 64, 0)
+    assert need >= L.asa_fwd_workspace_size(1, 2, 1024, 64, 0) + 2 * 1024 * 64 * 2
+    args[11], args[12] = FAKE, need
+    args[15] = MIS
+    assert L.asa_sparse_attn_fwd_train(*args) == asa.ASA_ERR_INVALID_ARG
+    args[15] = FAKE
+    args[8] = 96
+    assert L.asa_sparse_attn_fwd_train(*args) == asa.ASA_ERR_UNSUPPORTED
+    # backward: the asa_sparse_attn_bwd contract with o32 in place of o
+    bargs = [FAKE] * 10 + [1, 2, 1024, 64, 128, 0, None, 0] + [FAKE] * 3 + [None]
+    assert L.asa_sparse_attn_bwd_train(*bargs) == asa.ASA_ERR_WORKSPACE
+    bargs[15] = -1
+    assert L.asa_sparse_attn_bwd_train(*bargs) == asa.ASA_ERR_INVALID_ARG
+    bargs[15] = 0
+    bargs[3] = MIS
+    assert L.asa_sparse_attn_bwd_train(*bargs) == asa.ASA_ERR_INVALID_ARG
+    assert b"o32" in L.asa_last_error_string()

@@ -59,9 +59,9 @@ def test_autograd_equals_step_by_step():
     out.backward(x["dout"].cuda())
     qp, kp, vp = asa.asa_gilbert_permute3(q.detach(), k.detach(), v.detach(), wl.T, wl.Hg, wl.W)
     m = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
-    op, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, m)
+    op, lse, o32 = asa.asa_sparse_attn_fwd_train(qp, kp, vp, m)
     dop = asa.asa_gilbert_permute(x["dout"].cuda(), wl.T, wl.Hg, wl.W)
-    grads = asa.asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, m)
+    grads = asa.asa_sparse_attn_bwd_train(qp, kp, vp, o32, dop, lse, m)
     asa.asa_check_device_status()
     assert torch.equal(out.detach(), asa.asa_unpermute(op, wl.T, wl.Hg, wl.W))
     for t, gp in zip((q, k, v), grads):

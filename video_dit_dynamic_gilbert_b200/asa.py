@@ -41,7 +41,11 @@ _SIGNATURES = {
     "asa_global_pool": ([_vp, _vp] + [_c_int] * 5 + [_vp], _c_int),
     "asa_fwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
+    "asa_fwd_train_workspace_size": ([_c_int] * 5, _c_size),
+    "asa_sparse_attn_fwd_train": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp, _vp],
+                                  _c_int),
     "asa_bwd_workspace_size": ([_c_int] * 5, _c_size),
+    "asa_sparse_attn_bwd_train": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_sparse_attn_bwd": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4, _c_int),
     "asa_sparse_attn_bwd_d_from_o": ([_vp] * 10 + [_c_int] * 6 + [_vp, _c_size] + [_vp] * 4,
                                      _c_int),
@@ -310,6 +314,32 @@ def asa_sparse_attn_fwd(qp, kp, vp, mask: BlockMask, global_window: int = 0, wor
     return out, lse
 
 
+def fwd_train_workspace(B, H, N, d, global_window, device):
+    return _workspace(lib().asa_fwd_train_workspace_size(B, H, N, d, global_window), device)
+
+
+def asa_sparse_attn_fwd_train(qp, kp, vp, mask: BlockMask, global_window: int = 0,
+                              workspace=None, out=None, lse=None, out32=None, stream=None):
+    """The training forward: O [B, H, N, d] bf16, LSE [B, H, N] fp32 and the fp32 O
+    [B, H, N, d] that asa_sparse_attn_bwd_train takes D from (P V in fp16)."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp)):
+        _bf16_cuda(n_, t)
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = fwd_train_workspace(B, H, N, d, global_window, qp.device)
+    if out is None:
+        out = torch.empty_like(qp)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=qp.device)
+    if out32 is None:
+        out32 = torch.empty(qp.shape, dtype=torch.float32, device=qp.device)
+    _check(lib().asa_sparse_attn_fwd_train(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(mask.row_ptr),
+                                           _ptr(mask.col_idx), B, H, N, d, BLOCK, global_window,
+                                           _ptr(workspace), _ws_bytes(workspace), _ptr(out),
+                                           _ptr(lse), _ptr(out32), _stream(stream)))
+    return out, lse, out32
+
+
 def bwd_workspace(B, H, N, d, device, global_window: int = 0):
     return _workspace(lib().asa_bwd_workspace_size(B, H, N, d, global_window), device)
 
@@ -333,6 +363,31 @@ def asa_sparse_attn_bwd(qp, kp, vp, o, dout, lse, mask: BlockMask, global_window
               _ptr(mask.col_idx), _ptr(mask.col_ptr_t), _ptr(mask.row_idx_t), B, H, N, d, BLOCK,
               global_window, _ptr(workspace), _ws_bytes(workspace), *(_ptr(t) for t in outs),
               _stream(stream)))
+    return outs
+
+
+def asa_sparse_attn_bwd_train(qp, kp, vp, o32, dout, lse, mask: BlockMask,
+                              global_window: int = 0, workspace=None, outs=None, stream=None):
+    """dQ, dK, dV after asa_sparse_attn_fwd_train: D = rowsum(dO * O) from its fp32 O
+    (no pass of its own over the kept tiles); lse from the same forward."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp), ("dout", dout)):
+        _bf16_cuda(n_, t)
+    if o32.dtype != torch.float32 or not o32.is_cuda or not o32.is_contiguous():
+        raise ValueError("o32 must be a contiguous fp32 CUDA tensor")
+    if mask.col_ptr_t is None:
+        raise ValueError("the backward needs the transposed CSR (transposed=True)")
+    B, H, N, d = qp.shape
+    if tuple(o32.shape) != (B, H, N, d):
+        raise ValueError(f"o32 shape {tuple(o32.shape)} != {(B, H, N, d)}")
+    if workspace is None:
+        workspace = bwd_workspace(B, H, N, d, qp.device, global_window)
+    if outs is None:
+        outs = tuple(torch.empty_like(qp) for _ in range(3))
+    _check(lib().asa_sparse_attn_bwd_train(
+        _ptr(qp), _ptr(kp), _ptr(vp), _ptr(o32), _ptr(dout), _ptr(lse), _ptr(mask.row_ptr),
+        _ptr(mask.col_idx), _ptr(mask.col_ptr_t), _ptr(mask.row_idx_t), B, H, N, d, BLOCK,
+        global_window, _ptr(workspace), _ws_bytes(workspace), *(_ptr(t) for t in outs),
+        _stream(stream)))
     return outs
 
 
@@ -532,8 +587,11 @@ def asa_attention_host(q, k, v, T: int, Hg: int, W: int, tau: float, global_wind
 class ASAAttention(torch.autograd.Function):
     """ASA (or ASA_G) self-attention as a differentiable op on raster-layout q, k, v
     [B, N, H, d] bf16.  The mask is computed in the forward from q and k and is not
-    differentiated (the pages fix it for training as for inference); the backward is
-    asa_sparse_attn_bwd under that mask, its gradients unpermuted to raster layout."""
+    differentiated (the pages fix it for training as for inference); the backward runs
+    under that mask, its gradients unpermuted to raster layout.  Without query pruning
+    the forward is asa_sparse_attn_fwd_train and the backward asa_sparse_attn_bwd_train
+    (D from the fp32 O); d_from_o=True takes the inference forward and
+    asa_sparse_attn_bwd_d_from_o instead; with query_keep the pruned pair."""
 
     @staticmethod
     def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
@@ -545,13 +603,16 @@ class ASAAttention(torch.autograd.Function):
         qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W)
         mask = asa_estimate_mask(qp, kp, tau, transposed=True)
         prune = None
-        if query_keep is None:
+        o32 = None
+        if query_keep is None and not d_from_o:
+            op, lse, o32 = asa_sparse_attn_fwd_train(qp, kp, vp, mask, global_window=global_window)
+        elif query_keep is None:
             op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window)
         else:
             prune = asa_prune_queries(qp, query_keep, query_window)
             tmask = asa_prune_mask(mask, prune.pack)
             op, lse = asa_sparse_attn_fwd_pruned(prune, kp, vp, tmask, global_window=global_window)
-        ctx.save_for_backward(qp, kp, vp, op, lse)
+        ctx.save_for_backward(qp, kp, vp, op if o32 is None else o32, lse)
         ctx.mask, ctx.grid, ctx.global_window, ctx.prune = mask, (T, Hg, W), global_window, prune
         ctx.tmask = tmask if prune is not None else None
         ctx.d_from_o = d_from_o
@@ -562,9 +623,12 @@ class ASAAttention(torch.autograd.Function):
         qp, kp, vp, op, lse = ctx.saved_tensors
         T, Hg, W = ctx.grid
         dop = asa_gilbert_permute(dout.to(torch.bfloat16).contiguous(), T, Hg, W)
-        if ctx.prune is None:
+        if ctx.prune is None and not ctx.d_from_o:
+            grads = asa_sparse_attn_bwd_train(qp, kp, vp, op, dop, lse, ctx.mask,
+                                              global_window=ctx.global_window)
+        elif ctx.prune is None:
             grads = asa_sparse_attn_bwd(qp, kp, vp, op, dop, lse, ctx.mask,
-                                        global_window=ctx.global_window, d_from_o=ctx.d_from_o)
+                                        global_window=ctx.global_window, d_from_o=True)
         else:
             grads = asa_sparse_attn_bwd_pruned(ctx.prune, kp, vp, dop, lse, ctx.tmask,
                                                global_window=ctx.global_window)

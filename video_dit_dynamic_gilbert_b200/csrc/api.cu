@@ -431,6 +431,73 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
   return ASA_OK;
 }
 
+size_t asa_fwd_train_workspace_size(int B, int H, int N, int d, int global_window) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128) || global_window < 0) return 0;
+  size_t bytes = asa_fwd_workspace_size(B, H, N, d, global_window);
+  bytes += align256(static_cast<size_t>(B) * H * N * d * 2);  // fp16 V
+  if (global_window > 0) {
+    const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    bytes += align256(static_cast<size_t>(B) * H * G * d * 2);  // fp16 global V tokens
+  }
+  return bytes;
+}
+
+int asa_sparse_attn_fwd_train(const void* qp, const void* kp, const void* vp,
+                              const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N,
+                              int d, int block, int global_window, void* workspace,
+                              size_t ws_bytes, void* o, float* lse, float* o32, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(vp, "vp"));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(o, "o"));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  ASA_TRY(check_ptr(o32, "o32"));
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  const size_t need = asa_fwd_train_workspace_size(B, H, N, d, global_window);
+  ASA_TRY(check_ws(workspace, ws_bytes, need));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current();
+  unsigned int* err_word = nullptr;
+  cudaError_t e = device_error_word(&err_word);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  // workspace: launch order, [global K and V tokens,] fp16 V, [fp16 global V tokens]
+  char* base = static_cast<char*>(workspace);
+  const size_t nb = (static_cast<size_t>(N) + ASA_BLOCK - 1) / ASA_BLOCK;
+  int32_t* order = reinterpret_cast<int32_t*>(base);
+  size_t off = align256(static_cast<size_t>(B) * H * nb * sizeof(int32_t));
+  const void* kg = nullptr;
+  void* vg = nullptr;
+  size_t G = 0;
+  if (global_window > 0) {
+    G = (static_cast<size_t>(N) + global_window - 1) / global_window;
+    void* kgw = base + off;
+    off += align256(static_cast<size_t>(B) * H * G * d * 2);
+    vg = base + off;
+    off += align256(static_cast<size_t>(B) * H * G * d * 2);
+    e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, sms, s);
+    if (e == cudaSuccess) e = asa::launch_global_pool(vp, vg, B * H, N, d, global_window, sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    kg = kgw;
+  }
+  void* v16 = base + off;
+  off += align256(static_cast<size_t>(B) * H * N * d * 2);
+  e = asa::launch_f16_copy(vp, v16, static_cast<int64_t>(B) * H * N * d, err_word, sms, s);
+  void* vg16 = nullptr;
+  if (e == cudaSuccess && global_window > 0) {
+    vg16 = base + off;
+    e = asa::launch_f16_copy(vg, vg16, static_cast<int64_t>(B) * H * G * d, err_word, sms, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "fp16 copy launch");
+  e = asa::launch_fwd_tc_train(qp, kp, v16, row_ptr, col_idx, kg, vg16, order, B * H, N, d,
+                               global_window, o, lse, o32, err_word, s);
+  if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return ASA_OK;
+}
+
 size_t asa_bwd_workspace_size(int B, int H, int N, int d, int global_window) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128) || global_window < 0) return 0;
   return asa::bwd_tc_workspace_bytes(B * H, N, d, global_window);
@@ -440,11 +507,12 @@ static int bwd_impl(const void* qp, const void* kp, const void* vp, const void* 
                     const void* dout, const float* lse, const int32_t* row_ptr,
                     const int32_t* col_idx, const int32_t* col_ptr_t, const int32_t* row_idx_t,
                     int B, int H, int N, int d, int block, int global_window, void* workspace,
-                    size_t ws_bytes, void* dq, void* dk, void* dv, void* stream, bool d_from_o) {
+                    size_t ws_bytes, void* dq, void* dk, void* dv, void* stream, bool d_from_o,
+                    bool o_f32 = false) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_block(block, ASA_SAMPLES));
   const void* bf[] = {qp, kp, vp, o, dout, dq, dk, dv};
-  const char* names[] = {"qp", "kp", "vp", "o", "dout", "dq", "dk", "dv"};
+  const char* names[] = {"qp", "kp", "vp", o_f32 ? "o32" : "o", "dout", "dq", "dk", "dv"};
   for (int k = 0; k < 8; ++k) ASA_TRY(check_ptr(bf[k], names[k]));
   ASA_TRY(check_ptr(lse, "lse", false));
   ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
@@ -459,7 +527,7 @@ static int bwd_impl(const void* qp, const void* kp, const void* vp, const void* 
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
   e = asa::launch_bwd_tc(qp, kp, vp, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B * H, N,
                          d, global_window, workspace, dq, dk, dv, err_word, num_sms_current(),
-                         static_cast<cudaStream_t>(stream), d_from_o ? o : nullptr);
+                         static_cast<cudaStream_t>(stream), d_from_o ? o : nullptr, o_f32);
   if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return ASA_OK;
 }
@@ -482,6 +550,16 @@ int asa_sparse_attn_bwd_d_from_o(const void* qp, const void* kp, const void* vp,
                                  void* dk, void* dv, void* stream) {
   return bwd_impl(qp, kp, vp, o, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B, H, N, d,
                   block, global_window, workspace, ws_bytes, dq, dk, dv, stream, true);
+}
+
+int asa_sparse_attn_bwd_train(const void* qp, const void* kp, const void* vp, const float* o32,
+                              const void* dout, const float* lse, const int32_t* row_ptr,
+                              const int32_t* col_idx, const int32_t* col_ptr_t,
+                              const int32_t* row_idx_t, int B, int H, int N, int d, int block,
+                              int global_window, void* workspace, size_t ws_bytes, void* dq,
+                              void* dk, void* dv, void* stream) {
+  return bwd_impl(qp, kp, vp, o32, dout, lse, row_ptr, col_idx, col_ptr_t, row_idx_t, B, H, N, d,
+                  block, global_window, workspace, ws_bytes, dq, dk, dv, stream, true, true);
 }
 
 // ---------------------------------------------------------------- query pruning (BSA)
@@ -956,7 +1034,8 @@ int asa_check_device_status(void* stream) {
     cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
     if (word & 8u)
       return fail(ASA_ERR_INVALID_ARG,
-                  "backward: a Q or K value is out of fp16 range (|x| > 65504) (word 0x%x)", word);
+                  "a Q or K value (backward) or V value (training forward) is out of fp16 range "
+                  "(|x| > 65504) (word 0x%x)", word);
     if (word & 32u)
       return fail(ASA_ERR_INVALID_ARG,
                   "an index argument (CSR column, src_pos or src_row) is out of range (word 0x%x)",

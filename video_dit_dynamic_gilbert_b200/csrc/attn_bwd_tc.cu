@@ -860,11 +860,12 @@ __global__ void __launch_bounds__(256)
 
 size_t a256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// D = rowsum(dO * O) from the stored bf16 O (the opt-in approximate D): one warp per
-// row, fp32 accumulation; rows past N keep the 0 of bwd_prep.
-template <int D>
+// D = rowsum(dO * O) from a stored O: the bf16 O of the inference forward (the opt-in
+// approximate D) or the fp32 O of the training forward.  One warp per row, fp32
+// accumulation; rows past N keep the 0 of bwd_prep.
+template <int D, bool kF32>
 __global__ void __launch_bounds__(256)
-    d_from_o_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o,
+    d_from_o_kernel(const __nv_bfloat16* __restrict__ dout, const void* __restrict__ o,
                     int64_t rows, int N, int Np, float* __restrict__ Dvec) {
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
@@ -872,14 +873,24 @@ __global__ void __launch_bounds__(256)
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        row < rows; row += warps) {
     const __nv_bfloat16* a = dout + row * D + lane * E;
-    const __nv_bfloat16* b = o + row * D + lane * E;
     float acc = 0.f;
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
       const uint32_t ua = *reinterpret_cast<const uint32_t*>(a + e);
-      const uint32_t ub = *reinterpret_cast<const uint32_t*>(b + e);
-      acc = fmaf(__uint_as_float(ua << 16), __uint_as_float(ub << 16), acc);
-      acc = fmaf(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u), acc);
+      float b0, b1;
+      if constexpr (kF32) {
+        const float2 v = *reinterpret_cast<const float2*>(static_cast<const float*>(o) + row * D +
+                                                          lane * E + e);
+        b0 = v.x;
+        b1 = v.y;
+      } else {
+        const uint32_t ub = *reinterpret_cast<const uint32_t*>(
+            static_cast<const __nv_bfloat16*>(o) + row * D + lane * E + e);
+        b0 = __uint_as_float(ub << 16);
+        b1 = __uint_as_float(ub & 0xffff0000u);
+      }
+      acc = fmaf(__uint_as_float(ua << 16), b0, acc);
+      acc = fmaf(__uint_as_float(ua & 0xffff0000u), b1, acc);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -1066,6 +1077,13 @@ PrunedWs carve_pruned(void* base, size_t start, int BH, int N, int Ns, int d) {
 
 }  // namespace
 
+cudaError_t launch_f16_copy(const void* src, void* dst, int64_t n, unsigned int* err_word,
+                            int num_sms, cudaStream_t stream) {
+  f16_copy_kernel<<<num_sms * 8, 256, 0, stream>>>(static_cast<const uint4*>(src),
+                                                   static_cast<uint4*>(dst), n / 8, err_word);
+  return cudaGetLastError();
+}
+
 size_t bwd_tc_workspace_bytes(int BH, int N, int d, int global_window) {
   if (BH < 1 || N < 1 || global_window < 0) return 0;
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
@@ -1084,7 +1102,7 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk, void* dv,
                           unsigned int* err_word, int num_sms, cudaStream_t stream,
-                          const void* o_for_d) {
+                          const void* o_for_d, bool o_f32) {
   const int nb = (N + kBlock - 1) / kBlock;
   const int Np = nb * kBlock;
   const int gw = global_window;
@@ -1105,11 +1123,14 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
     const int64_t rows = static_cast<int64_t>(BH) * N;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>((rows + 7) / 8, num_sms * 16));
     const auto* a = static_cast<const __nv_bfloat16*>(dout);
-    const auto* b = static_cast<const __nv_bfloat16*>(o_for_d);
-    if (d == 128)
-      d_from_o_kernel<128><<<grid, 256, 0, stream>>>(a, b, rows, N, Np, ws.Dvec);
+    if (o_f32 && d == 128)
+      d_from_o_kernel<128, true><<<grid, 256, 0, stream>>>(a, o_for_d, rows, N, Np, ws.Dvec);
+    else if (o_f32)
+      d_from_o_kernel<64, true><<<grid, 256, 0, stream>>>(a, o_for_d, rows, N, Np, ws.Dvec);
+    else if (d == 128)
+      d_from_o_kernel<128, false><<<grid, 256, 0, stream>>>(a, o_for_d, rows, N, Np, ws.Dvec);
     else
-      d_from_o_kernel<64><<<grid, 256, 0, stream>>>(a, b, rows, N, Np, ws.Dvec);
+      d_from_o_kernel<64, false><<<grid, 256, 0, stream>>>(a, o_for_d, rows, N, Np, ws.Dvec);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;

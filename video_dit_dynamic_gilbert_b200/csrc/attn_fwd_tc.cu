@@ -21,7 +21,12 @@
 //               the two partial results are merged (max, scaled sums) and O / l is
 //               written as bf16 rows with the natural-log LSE.
 // TMEM: S buffers at columns [0,128) and [128,256), O_0 at [256,256+D), O_1 at
-// [384,384+D).  Every wait is bounded: on expiry the kernel sets the device error word,
+// [384,384+D).
+// Training variant (kTrain): P is packed as fp16 and multiplies an fp16 copy of V (a
+// kind::f16 MMA takes A and B of one type), and the merged fp32 O is also written out.
+// P <= 2^8 by the rescale rule, so fp16 holds it; its 11 significant bits put ~8x less
+// rounding error on O than bf16's 8, which is what lets the backward take
+// D = rowsum(dO o O) from that fp32 O instead of a pass of its own.  Every wait is bounded: on expiry the kernel sets the device error word,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
@@ -89,7 +94,7 @@ __device__ __forceinline__ TileSrc tile_src(int j, int nfine, const int32_t* col
 // kPruned: the query tiles are packed tiles of pruned queries (Nq rows per head).
 // Entry e of the tile's CSR row is seen only by the 32-row lane quarters q with bit q
 // of quarters[e] set; the other quarters' rows give that key tile probability 0.
-template <int D, int NST, bool kPruned>
+template <int D, int NST, bool kPruned, bool kTrain>
 __global__ void __launch_bounds__(kFwdTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKg,
@@ -97,7 +102,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
                   const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ quarters,
                   const int32_t* __restrict__ order, int N, int Nq, int nb, int G, float gbias2,
                   float c2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                  unsigned int* __restrict__ err_word, long long wait_limit) {
+                  float* __restrict__ o32, unsigned int* __restrict__ err_word,
+                  long long wait_limit) {
   using L = FwdTcLayout<D, NST>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -200,7 +206,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idPV = tc::idesc_bf16(128, D, false, true);
+      constexpr uint32_t idPV =
+          kTrain ? tc::idesc_f16(128, D, false, true) : tc::idesc_bf16(128, D, false, true);
       // Descriptors are built once; an offset of `o` bytes into a tile adds o >> 4 to
       // the start-address field (all tiles lie below 256 KB, so it never carries).
       const uint64_t dQ = tc::sdesc_sw128(base + L::kQ, 16, 1024);
@@ -326,7 +333,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       const bool any_need = __any_sync(0xffffffffu, need) != 0;
       const float alpha = need ? (m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new)) : 1.f;
       if (need) m_ref = m_new;
-      // P = exp2(s c2 + bias - m) packed to bf16 pairs (masked columns give exp2(-inf) = 0)
+      // P = exp2(s c2 + bias - m) packed to bf16 pairs, fp16 in training (masked columns
+      // give exp2(-inf) = 0)
       const float off = bias - (m_ref == -INFINITY ? 0.f : m_ref);
       uint32_t p[64];
       const uint64_t c2x2 = f2_pack(c2, c2), offx2 = f2_pack(off, off);
@@ -346,7 +354,7 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
           bb = fast_exp2(xb);
         }
         rs = f2_add(rs, f2_pack(a, bb));
-        p[k] = pack_bf16(a, bb);
+        p[k] = kTrain ? pack_f16(a, bb) : pack_bf16(a, bb);
       }
       float rsa, rsb;
       f2_unpack(rs, rsa, rsb);
@@ -408,7 +416,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
     // warpgroup w writes columns [D/2 w, D/2 w + D/2) of its rows
     const int q = q0 + row;
-    __nv_bfloat16* orow = o + (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
+    const int64_t orow_off = (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
+    __nv_bfloat16* orow = o + orow_off;
     const bool h0 = __all_sync(0xffffffffu, has_0) != 0 || __any_sync(0xffffffffu, has_0) != 0;
     const bool h1 = __any_sync(0xffffffffu, has_1) != 0;
 #pragma unroll
@@ -444,6 +453,11 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
           pk.z = pack_bf16(x[4], x[5]);
           pk.w = pack_bf16(x[6], x[7]);
           *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v) = pk;
+          if constexpr (kTrain) {
+            float4* o32row = reinterpret_cast<float4*>(o32 + orow_off + 32 * c + 8 * v);
+            o32row[0] = make_float4(x[0], x[1], x[2], x[3]);
+            o32row[1] = make_float4(x[4], x[5], x[6], x[7]);
+          }
         }
       }
     }
@@ -557,22 +571,22 @@ cudaError_t launch_lpt_order(const int32_t* ptr, int BH, int nrows, int maxc, in
 namespace {
 
 // Nq query rows per head in nb query tiles (N, ceil(N/128) without pruning).
-template <int D, int NST, bool kPruned>
+template <int D, int NST, bool kPruned, bool kTrain>
 cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int32_t* col_idx,
                       const uint8_t* quarters, int32_t* order, int BH, int N, int Nq, int G,
-                      float gbias2, void* o, float* lse, unsigned int* err_word,
+                      float gbias2, void* o, float* lse, float* o32, unsigned int* err_word,
                       cudaStream_t stream) {
   using L = FwdTcLayout<D, NST>;
   const int nb = (Nq + kBlock - 1) / kBlock;
   const float c2 = kLog2e / sqrtf(static_cast<float>(D));
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST, kPruned>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D, NST, kPruned, kTrain>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   // the register split inside the kernel assumes exactly kLaunchRegs per thread at launch
   static int regs_checked = 0;
   if (regs_checked == 0) {
     cudaFuncAttributes fa{};
-    e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<D, NST, kPruned>);
+    e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<D, NST, kPruned, kTrain>);
     if (e != cudaSuccess) return e;
     regs_checked = fa.numRegs == kLaunchRegs ? 1 : -1;
   }
@@ -582,36 +596,39 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   // a row holds at most one entry per key block
   e = launch_lpt_order(row_ptr, BH, nb, (N + kBlock - 1) / kBlock, order, stream);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<D, NST, kPruned><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
+  fwd_tc_kernel<D, NST, kPruned, kTrain><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, quarters, order, N, Nq, nb,
-      G, gbias2, c2, static_cast<__nv_bfloat16*>(o), lse, err_word, limit);
+      G, gbias2, c2, static_cast<__nv_bfloat16*>(o), lse, o32, err_word, limit);
   return cudaGetLastError();
 }
 
-template <bool kPruned>
+// kTrain: vp and vg are the fp16 copies of V and of the global V tokens.
+template <bool kPruned, bool kTrain = false>
 cudaError_t launch_fwd_any(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
                            const int32_t* col_idx, const uint8_t* quarters, const void* kg,
                            const void* vg, int32_t* order, int BH, int N, int Nq, int d,
-                           int global_window, void* o, float* lse, unsigned int* err_word,
-                           cudaStream_t stream) {
+                           int global_window, void* o, float* lse, float* o32,
+                           unsigned int* err_word, cudaStream_t stream) {
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
   const float gbias2 = global_window > 0 ? log2f(static_cast<float>(global_window)) : 0.f;
+  const CUtensorMapDataType vtype =
+      kTrain ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap maps[5];
   if (!make_map(&maps[0], qp, BH, Nq, d) || !make_map(&maps[1], kp, BH, N, d) ||
-      !make_map(&maps[2], vp, BH, N, d))
+      !make_map_dtype(&maps[2], vp, BH, N, d, vtype))
     return cudaErrorInvalidValue;
   if (G > 0) {
-    if (!make_map(&maps[3], kg, BH, G, d) || !make_map(&maps[4], vg, BH, G, d))
+    if (!make_map(&maps[3], kg, BH, G, d) || !make_map_dtype(&maps[4], vg, BH, G, d, vtype))
       return cudaErrorInvalidValue;
   } else {
     maps[3] = maps[1];
     maps[4] = maps[2];
   }
   if (d == 128)
-    return launch_tc<128, 3, kPruned>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G,
-                                      gbias2, o, lse, err_word, stream);
-  return launch_tc<64, 6, kPruned>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G, gbias2,
-                                   o, lse, err_word, stream);
+    return launch_tc<128, 3, kPruned, kTrain>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq,
+                                              G, gbias2, o, lse, o32, err_word, stream);
+  return launch_tc<64, 6, kPruned, kTrain>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G,
+                                           gbias2, o, lse, o32, err_word, stream);
 }
 
 }  // namespace
@@ -621,7 +638,16 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
                           int BH, int N, int d, int global_window, void* o, float* lse,
                           unsigned int* err_word, cudaStream_t stream) {
   return launch_fwd_any<false>(qp, kp, vp, row_ptr, col_idx, nullptr, kg, vg, order, BH, N, N, d,
-                               global_window, o, lse, err_word, stream);
+                               global_window, o, lse, nullptr, err_word, stream);
+}
+
+cudaError_t launch_fwd_tc_train(const void* qp, const void* kp, const void* vp16,
+                                const int32_t* row_ptr, const int32_t* col_idx, const void* kg,
+                                const void* vg16, int32_t* order, int BH, int N, int d,
+                                int global_window, void* o, float* lse, float* o32,
+                                unsigned int* err_word, cudaStream_t stream) {
+  return launch_fwd_any<false, true>(qp, kp, vp16, row_ptr, col_idx, nullptr, kg, vg16, order, BH,
+                                     N, N, d, global_window, o, lse, o32, err_word, stream);
 }
 
 cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp,
@@ -631,7 +657,7 @@ cudaError_t launch_fwd_tc_pruned(const void* q_s, const void* kp, const void* vp
                                  void* o_s, float* lse_s, unsigned int* err_word,
                                  cudaStream_t stream) {
   return launch_fwd_any<true>(q_s, kp, vp, tile_ptr, tile_col, quarters, kg, vg, order, BH, N, Ns,
-                              d, global_window, o_s, lse_s, err_word, stream);
+                              d, global_window, o_s, lse_s, nullptr, err_word, stream);
 }
 
 }  // namespace asa

@@ -61,6 +61,14 @@ cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const 
                           int BH, int N, int d, int global_window, void* o, float* lse,
                           unsigned int* err_word, cudaStream_t stream);
 
+// Training forward: PV with fp16 P and the fp16 copies vp16, vg16 of V and of the
+// global V tokens; writes O (bf16), LSE and the fp32 O.
+cudaError_t launch_fwd_tc_train(const void* qp, const void* kp, const void* vp16,
+                                const int32_t* row_ptr, const int32_t* col_idx, const void* kg,
+                                const void* vg16, int32_t* order, int BH, int N, int d,
+                                int global_window, void* o, float* lse, float* o32,
+                                unsigned int* err_word, cudaStream_t stream);
+
 // Launch order of the rows of a CSR (ptr[BH * nrows + 1], global offsets): heads in
 // order, inside each head the rows with the most entries first; maxc bounds a row's
 // entry count (the number of key blocks).
@@ -76,7 +84,12 @@ cudaError_t launch_bwd_tc(const void* qp, const void* kp, const void* vp, const 
                           const int32_t* col_ptr_t, const int32_t* row_idx_t, int BH, int N,
                           int d, int global_window, void* workspace, void* dq, void* dk,
                           void* dv, unsigned int* err_word, int num_sms, cudaStream_t stream,
-                          const void* o_for_d = nullptr);
+                          const void* o_for_d = nullptr, bool o_f32 = false);
+
+// fp16 copy of n bf16 elements (n a multiple of 8); a value beyond fp16 range ORs 8
+// into the device error word
+cudaError_t launch_f16_copy(const void* src, void* dst, int64_t n, unsigned int* err_word,
+                            int num_sms, cudaStream_t stream);
 
 // Gilbert gather from / scatter into per-rank token chunks: chunk s holds the rows
 // [B][tok.off[s+1] - tok.off[s]][H][d] of rank s's tokens, chunks back to back (the
