@@ -293,15 +293,18 @@ def _near_threshold_rows(p_imp, tau, eps=1e-4, gap=1e-6):
 
 class _Timer:
     """Per-call CUDA-event times on one stream: median and min over `reps` calls after
-    `warm` untimed ones; `flush` (an L2-sized write) runs before each call, outside its
-    events."""
+    `warm` untimed ones; `flush` runs before each call, outside its events.  The flush
+    reads a buffer twice the size of L2: it evicts every line (and writes back, before
+    the timed call, whatever the previous call left dirty) while leaving only clean
+    lines behind, so that the timed call is not charged for someone else's
+    write-back (a flush that writes the buffer would add up to 126 MB of it)."""
 
     def __init__(self, torch, stream, flush_bytes=256 << 20):
         self.torch, self.stream = torch, stream
-        self.buf = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+        self.buf = torch.ones(flush_bytes // 4, dtype=torch.int32, device="cuda")
 
     def flush(self):
-        self.buf.fill_(1)
+        self.sink = self.buf.sum()
 
     def __call__(self, fn, reps=20, warm=5, flush=False):
         torch = self.torch
@@ -578,6 +581,11 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--report", metavar="PATH", default=None,
                     help="run the full measurement set on one GPU, write it to PATH as JSON")
+    ap.add_argument("--no-launch-count", action="store_true",
+                    help="skip the CUPTI count of the step's kernels (for runs under ncu)")
+    ap.add_argument("--only", choices=["bwd_train"], default=None,
+                    help="time one stage alone on the workload (training forward once, then "
+                         "--steps training backward calls) and print its JSON line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -588,6 +596,9 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args, wl)
+        return
+    if args.only == "bwd_train":
+        run_bwd_train_only(args, wl)
         return
 
     import torch
@@ -681,7 +692,8 @@ def main():
                      "frac_of_sustained": achieved / sustained},
         "clocks": clk,
     }
-    per_step, names = count_launches(torch, step)
+    per_step, names = ((None, "not counted (--no-launch-count)") if args.no_launch_count
+                       else count_launches(torch, step))
     result["gpu_launches"] = per_step * args.steps if per_step is not None else None
     result["gpu_launches_how"] = (f"{per_step} kernels of this library per step, counted by "
                                   f"CUPTI (torch.profiler) over one untimed step, x steps"
@@ -757,6 +769,43 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_bwd_train_only(args, wl):
+    """The training backward alone: Gilbert permute and mask of the workload, the
+    training forward once, then `warmup` untimed and `steps` timed backward calls
+    (CUDA events on the stream); one JSON line with its ms and effective TFLOP/s."""
+    import torch
+    from inputs import make_inputs
+    from video_dit_dynamic_gilbert_b200 import asa
+    dev = torch.device("cuda", 0)
+    x = make_inputs(wl, with_dout=True)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "dout"))
+    qp, kp, vp, dop = (asa.asa_gilbert_permute(t, wl.T, wl.Hg, wl.W) for t in (q, k, v, do))
+    m = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
+    o, lse, o32 = asa.asa_sparse_attn_fwd_train(qp, kp, vp, m, global_window=wl.global_window)
+    B, H, N, d = qp.shape
+    ws = asa.bwd_workspace(B, H, N, d, dev, wl.global_window)
+    outs = tuple(torch.empty_like(qp) for _ in range(3))
+    call = lambda: asa.asa_sparse_attn_bwd_train(qp, kp, vp, o32, dop, lse, m,
+                                                 global_window=wl.global_window, workspace=ws,
+                                                 outs=outs)
+    for _ in range(args.warmup):
+        call()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    asa.asa_check_device_status()
+    ms = a.elapsed_time(b) / args.steps
+    flops, _, _ = _kept_tile_flops(m.row_ptr.cpu().numpy(), m.col_idx.cpu().numpy(), B, H, N, d)
+    print(json.dumps({"stage": "bwd_train", "workload": wl.name, "ms": ms,
+                      "effective_tflops": 2.5 * flops / ms / 1e9, "steps": args.steps,
+                      "warmup": args.warmup}))
 
 
 def extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream):

@@ -385,6 +385,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t dsum2 = f2_pack(0.f, 0.f);
     for (int t = 0; t < n; ++t) {
       const uint32_t tS = trow + 128u * (t & 1) + 64u * w;
+      // global tokens carry + ln(n) (log2(n) in these units); with query pruning a
+      // warp whose rows do not keep key block cols[t] gives it probability 0.  Key
+      // columns past N (the ragged last block) or past G get no weight.  The CSR reads
+      // come before the wait for S, so their latency is not added after it.
+      const bool glob = t >= nfine;
+      const bool mine = !kPruned || glob || ((qbits[t] >> quarter) & 1u);
+      const float off = mine ? nl2 + (glob ? gbias2 : 0.f) : -INFINITY;
+      const int nvalid = (glob ? min(kBlock, G - (t - nfine) * kBlock)
+                               : min(kBlock, N - cols[t] * kBlock)) - 64 * w;
       if (!wait_warp(br.s_full(t & 1), (t >> 1) & 1)) {
         failed = true;
         break;
@@ -397,15 +406,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::tmem_wait_ld_dep32(s + 32);
       if (kDPass) warp_arrive(br.ds_full(t & 1), lane);
       float p[64];
-      // global tokens carry + ln(n) (log2(n) in these units); with query pruning a
-      // warp whose rows do not keep key block cols[t] gives it probability 0
-      const bool glob = t >= nfine;
-      const bool mine = !kPruned || glob || ((qbits[t] >> quarter) & 1u);
-      const float off = mine ? nl2 + (glob ? gbias2 : 0.f) : -INFINITY;
       exp2_64(s, c2, [&](int) { return off; }, p);
-      // key columns past N (the ragged last block) or past G get no weight
-      const int nvalid = (glob ? min(kBlock, G - (t - nfine) * kBlock)
-                               : min(kBlock, N - cols[t] * kBlock)) - 64 * w;
       if (nvalid < 64) {
 #pragma unroll
         for (int k = 0; k < 64; ++k)
@@ -692,6 +693,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::tmem_wait_ld_dep32(s + 32);
       float p[64];
       exp2_64(s, c2, [&](int k) { return off[k]; }, p);  // query rows past N: lse2 = +inf, P = 0
+      float4 dq4[16];  // the query tile's D, loaded while P^T is stored and dP^T awaited
+#pragma unroll
+      for (int c = 0; c < 16; ++c) dq4[c] = __ldg(dvv + c);
       uint32_t pk[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) pk[k] = pack_bf16(p[2 * k], p[2 * k + 1]);
@@ -712,7 +716,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t ds[32];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 v = __ldg(dvv + c);
+        const float4 v = dq4[c];
         ds[2 * c] = pack_f16(p[4 * c] * (__uint_as_float(dp[4 * c]) - v.x),
                              p[4 * c + 1] * (__uint_as_float(dp[4 * c + 1]) - v.y));
         ds[2 * c + 1] = pack_f16(p[4 * c + 2] * (__uint_as_float(dp[4 * c + 2]) - v.z),

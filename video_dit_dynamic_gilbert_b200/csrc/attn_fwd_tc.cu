@@ -286,14 +286,17 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     float m_ref = -INFINITY, l = 0.f;
     int it = 0;  // tiles of this stream done
     for (int j = w; j < ntile; j += 2, ++it) {
+      // the tile's key block (and, with pruning, its lane-quarter bits) are read before
+      // the wait for S, so that their load latency is not added after it
+      const TileSrc t = tile_src(j, nfine, cols, N, G);
+      const bool skip = kPruned && !t.global && ((quarters[rbeg + j] >> quarter) & 1u) == 0u;
       if (!wait_warp(s_full(w), it & 1)) {
         failed = true;
         break;
       }
       tc::fence_after();
-      const TileSrc t = tile_src(j, nfine, cols, N, G);
       if constexpr (kPruned) {
-        if (!t.global && ((quarters[rbeg + j] >> quarter) & 1u) == 0u) {
+        if (skip) {
           // these rows do not keep key block cols[j]: P = 0, running max and sum unchanged
           uint32_t z[16];
 #pragma unroll
