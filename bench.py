@@ -385,6 +385,9 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
         kg = torch.empty((B, H, G, d), dtype=torch.bfloat16, device=dev)
         hbm_stage("pool_K", lambda: asa.asa_global_pool(kp, gw, out=kg),
                   tensor_bytes + B * H * G * d * 2)
+        vg = torch.empty_like(kg)
+        hbm_stage("pool_KV", lambda: asa.asa_global_pool_kv(kp, vp, gw, outs=(kg, vg)),
+                  2 * (tensor_bytes + B * H * G * d * 2))
         flops += 4 * d * N * G * B * H
     r["effective_flops"] = flops
     r["attn_fwd"] = timer(lambda: asa.asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=gw,
@@ -737,7 +740,9 @@ def main():
                      "call": "asa_attention_host (pinned host buffers, head chunks pipelined)"}
 
     if not args.no_extras:
+        xclocks = ClockSampler(local)
         result["extras"] = extras(asa, wl, q, k, v, qp, kp, vp, mask, dev, stream)
+        result["extras"]["clocks"] = xclocks.stop()
         # the host-buffer call by head chunk, and the unpipelined sequence (copy Q, K, V
         # in, device call, copy O out) for comparison
         by_chunk = {}

@@ -178,6 +178,11 @@ int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d
  */
 int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n, void* stream);
 
+/* asa_global_pool of K (into kg) and V (into vg) in one launch, as the ASA_G forward and
+ * backward build their global tokens.  Same layouts and errors as asa_global_pool. */
+int asa_global_pool_kv(const void* kp, const void* vp, void* kg, void* vg, int B, int H, int N,
+                       int d, int n, void* stream);
+
 /* Workspace bytes of asa_sparse_attn_fwd: the launch order of the query blocks
  * (longest kept list first), plus the global tokens for ASA_G. */
 size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window);

@@ -324,3 +324,12 @@ def test_training_pair_rejects(L):
     bargs[3] = MIS
     assert L.asa_sparse_attn_bwd_train(*bargs) == asa.ASA_ERR_INVALID_ARG
     assert b"o32" in L.asa_last_error_string()
+
+
+def test_global_pool_kv_rejects(L):
+    assert L.asa_global_pool_kv(FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 64, 0, None) == \
+        asa.ASA_ERR_INVALID_ARG
+    assert L.asa_global_pool_kv(FAKE, MIS, FAKE, FAKE, 1, 2, 1024, 64, 64, None) == \
+        asa.ASA_ERR_INVALID_ARG
+    assert L.asa_global_pool_kv(FAKE, FAKE, FAKE, FAKE, 1, 2, 1024, 96, 64, None) == \
+        asa.ASA_ERR_UNSUPPORTED

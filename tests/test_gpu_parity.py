@@ -200,6 +200,18 @@ def test_global_pool(name, n):
             assert (got[bb, h] == exp).mean() > 0.99
 
 
+@pytest.mark.parametrize("name,n", [("tiny", 64), ("one-ragged-block", 7), ("tail-lt-k", 1),
+                                    ("multi-tile", 200)])
+def test_global_pool_kv_one_launch(name, n):
+    """K and V pooled in one launch equal the two single-tensor launches bit for bit."""
+    wl, x, perm, ref, *_ = setup_case(name)
+    kp = torch.from_numpy(ref["k"]).to(torch.bfloat16).cuda()
+    vp = torch.from_numpy(ref["v"]).to(torch.bfloat16).cuda()
+    kg, vg = asa.asa_global_pool_kv(kp, vp, n)
+    assert torch.equal(kg.view(torch.int16), asa.asa_global_pool(kp, n).view(torch.int16))
+    assert torch.equal(vg.view(torch.int16), asa.asa_global_pool(vp, n).view(torch.int16))
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_backward_with_oracle_mask(name):
     wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "asa_build_mask": ([_vp, _c_int, _c_int, _c_int, _c_float, _vp, _c_size] + [_vp] * 6, _c_int),
     "asa_estimate_mask": ([_vp, _vp] + [_c_int] * 6 + [_c_float, _vp, _c_size] + [_vp] * 6, _c_int),
     "asa_global_pool": ([_vp, _vp] + [_c_int] * 5 + [_vp], _c_int),
+    "asa_global_pool_kv": ([_vp] * 4 + [_c_int] * 5 + [_vp], _c_int),
     "asa_fwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
     "asa_fwd_train_workspace_size": ([_c_int] * 5, _c_size),
@@ -289,6 +290,22 @@ def asa_global_pool(xp: torch.Tensor, n: int, out=None, stream=None):
         out = torch.empty((B, H, G, d), dtype=xp.dtype, device=xp.device)
     _check(lib().asa_global_pool(_ptr(xp), _ptr(out), B, H, N, d, n, _stream(stream)))
     return out
+
+
+def asa_global_pool_kv(kp: torch.Tensor, vp: torch.Tensor, n: int, outs=None, stream=None):
+    """The global tokens of K and V in one launch: (Kg, Vg) [B, H, ceil(N/n), d] bf16."""
+    _bf16_cuda("kp", kp)
+    _bf16_cuda("vp", vp)
+    if kp.shape != vp.shape:
+        raise ValueError("kp and vp must have the same shape")
+    B, H, N, d = kp.shape
+    G = -(-N // n)
+    if outs is None:
+        outs = tuple(torch.empty((B, H, G, d), dtype=torch.bfloat16, device=kp.device)
+                     for _ in range(2))
+    _check(lib().asa_global_pool_kv(_ptr(kp), _ptr(vp), _ptr(outs[0]), _ptr(outs[1]), B, H, N, d,
+                                    n, _stream(stream)))
+    return outs
 
 
 def fwd_workspace(B, H, N, d, global_window, device):

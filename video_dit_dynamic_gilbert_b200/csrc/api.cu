@@ -367,6 +367,20 @@ int asa_estimate_mask(const void* qp, const void* kp, int B, int H, int N, int d
                          stream);
 }
 
+int asa_global_pool_kv(const void* kp, const void* vp, void* kg, void* vg, int B, int H, int N,
+                       int d, int n, void* stream) {
+  ASA_TRY(check_common(B, H, N, d));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(vp, "vp"));
+  ASA_TRY(check_ptr(kg, "kg"));
+  ASA_TRY(check_ptr(vg, "vg"));
+  if (n < 1) return fail(ASA_ERR_INVALID_ARG, "global window n=%d must be >= 1", n);
+  cudaError_t e = asa::launch_global_pool(kp, kg, B * H, N, d, n, num_sms_current(),
+                                          static_cast<cudaStream_t>(stream), vp, vg);
+  if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+  return ASA_OK;
+}
+
 int asa_global_pool(const void* xp, void* xg, int B, int H, int N, int d, int n, void* stream) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_ptr(xp, "xp"));
@@ -415,9 +429,8 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
     char* base = static_cast<char*>(workspace) + align256(static_cast<size_t>(B) * H * nb * sizeof(int32_t));
     void* kgw = base;
     void* vgw = base + align256(static_cast<size_t>(B) * H * G * d * 2);
-    cudaError_t e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, num_sms_current(), s);
-    if (e == cudaSuccess)
-      e = asa::launch_global_pool(vp, vgw, B * H, N, d, global_window, num_sms_current(), s);
+    cudaError_t e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, num_sms_current(),
+                                            s, vp, vgw);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
     kg = kgw;
     vg = vgw;
@@ -478,8 +491,7 @@ int asa_sparse_attn_fwd_train(const void* qp, const void* kp, const void* vp,
     off += align256(static_cast<size_t>(B) * H * G * d * 2);
     vg = base + off;
     off += align256(static_cast<size_t>(B) * H * G * d * 2);
-    e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, sms, s);
-    if (e == cudaSuccess) e = asa::launch_global_pool(vp, vg, B * H, N, d, global_window, sms, s);
+    e = asa::launch_global_pool(kp, kgw, B * H, N, d, global_window, sms, s, vp, vg);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
     kg = kgw;
   }
@@ -706,8 +718,7 @@ int asa_sparse_attn_fwd_pruned(const void* q_s, const void* kp, const void* vp,
     const size_t G = (static_cast<size_t>(N) + global_window - 1) / global_window;
     void* kgw = p;
     void* vgw = p + align256(static_cast<size_t>(BH) * G * d * 2);
-    e = asa::launch_global_pool(kp, kgw, BH, N, d, global_window, num_sms_current(), s);
-    if (e == cudaSuccess) e = asa::launch_global_pool(vp, vgw, BH, N, d, global_window, num_sms_current(), s);
+    e = asa::launch_global_pool(kp, kgw, BH, N, d, global_window, num_sms_current(), s, vp, vgw);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
     kg = kgw;
     vg = vgw;

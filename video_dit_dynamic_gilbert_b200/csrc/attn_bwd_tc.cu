@@ -1035,8 +1035,7 @@ bool make_bwd_maps(CUtensorMap* maps, const BwdWs& ws, const void* dout, const v
 // the forward's global tokens, recomputed: mean-pooled K and V, Kg also in fp16
 cudaError_t global_tokens(const void* kp, const void* vp, const BwdWs& ws, int BH, int N, int d,
                           int gw, int G, unsigned int* err_word, int num_sms, cudaStream_t stream) {
-  cudaError_t e = launch_global_pool(kp, ws.kg, BH, N, d, gw, num_sms, stream);
-  if (e == cudaSuccess) e = launch_global_pool(vp, ws.vg, BH, N, d, gw, num_sms, stream);
+  cudaError_t e = launch_global_pool(kp, ws.kg, BH, N, d, gw, num_sms, stream, vp, ws.vg);
   if (e != cudaSuccess) return e;
   f16_copy_kernel<<<num_sms * 8, 256, 0, stream>>>(static_cast<const uint4*>(ws.kg),
                                                    static_cast<uint4*>(ws.kg16),

@@ -17,13 +17,22 @@ constexpr int kPoolUnroll = 8;
 // chunk c % (D/8) = tid % (D/8), since 128 is a multiple of D/8).  Column sums are then
 // added across the lanes of a warp that share a column chunk (xor shuffles over the
 // lane bits above log2(D/8)) and across the four warps in shared memory.
+// Blocks [0, BH G) pool xp into xg; with a second tensor (xp2 non-null), blocks
+// [BH G, 2 BH G) pool xp2 into xg2 in the same launch.
 __global__ void __launch_bounds__(kPoolThreads)
-    pool_kernel(const __nv_bfloat16* __restrict__ xp, __nv_bfloat16* __restrict__ xg, int N,
-                int D, int n, int G) {
+    pool_kernel(const __nv_bfloat16* __restrict__ xp, __nv_bfloat16* __restrict__ xg,
+                const __nv_bfloat16* __restrict__ xp2, __nv_bfloat16* __restrict__ xg2, int BH,
+                int N, int D, int n, int G) {
   __shared__ float red[kPoolThreads / 32][16][8];
   const int CH = D / 8;
-  const int gi = blockIdx.x % G;
-  const int64_t bh = blockIdx.x / G;
+  int64_t blk = blockIdx.x;
+  if (blk >= static_cast<int64_t>(BH) * G) {
+    blk -= static_cast<int64_t>(BH) * G;
+    xp = xp2;
+    xg = xg2;
+  }
+  const int gi = static_cast<int>(blk % G);
+  const int64_t bh = blk / G;
   const int beg = gi * n, end = min(N, beg + n);
   const int nchunk = (end - beg) * CH;
   const uint4* src = reinterpret_cast<const uint4*>(xp + (bh * N + beg) * D);
@@ -77,13 +86,14 @@ __global__ void __launch_bounds__(kPoolThreads)
 }  // namespace
 
 cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, int n, int num_sms,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const void* xp2, void* xg2) {
   (void)num_sms;
   const int G = (N + n - 1) / n;
-  const int64_t blocks = static_cast<int64_t>(BH) * G;  // one per window
+  const int64_t blocks = static_cast<int64_t>(BH) * G * (xp2 != nullptr ? 2 : 1);  // one per window
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
   pool_kernel<<<static_cast<unsigned>(blocks), kPoolThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(xp), static_cast<__nv_bfloat16*>(xg), N, d, n, G);
+      static_cast<const __nv_bfloat16*>(xp), static_cast<__nv_bfloat16*>(xg),
+      static_cast<const __nv_bfloat16*>(xp2), static_cast<__nv_bfloat16*>(xg2), BH, N, d, n, G);
   return cudaGetLastError();
 }
 

@@ -54,7 +54,8 @@ cudaError_t launch_build_mask_stat(const float* p_imp, int BH, int nb, double z,
                                    cudaStream_t stream);
 
 cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, int n, int num_sms,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const void* xp2 = nullptr,
+                               void* xg2 = nullptr);
 
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
                           const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
