@@ -251,13 +251,18 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
         for (int ks = 0; ks < kBlock / 16; ++ks)
           tc::umma_ts(tO, tP + 8u * ks, vst + ((ks * 2048u) >> 4), idPV,
                       (j >= 2 || ks > 0) ? 1u : 0u);
+        // the stream's next S goes into the buffer P_j just left (in issue order); the
+        // commits follow both MMA groups (each costs the issuing thread, and a commit
+        // tracks every MMA issued before it).  MMAs of one thread complete in order, so
+        // the S_{j+2} that the stream waits for next also tells it that PV_j is done;
+        // o_done is committed only after a stream's last PV, for the epilogue.
+        if (j + 2 < ntile) issue_s(j + 2);
         tc::umma_commit(v_empty(j % NST));
-        tc::umma_commit(o_done(b));
-        // the stream's next S goes into the buffer P_j just left (in issue order)
         if (j + 2 < ntile) {
-          issue_s(j + 2);
           tc::umma_commit(s_full(b));
           tc::umma_commit(k_empty((j + 2) % NST));
+        } else {
+          tc::umma_commit(o_done(b));
         }
       }
       failed = !ok;
@@ -363,12 +368,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       f2_unpack(rs, rsa, rsb);
       l = l * alpha + (rsa + rsb);
       if (it > 0) {
-        // this stream's previous PV is done: O may be rescaled
-        if (!wait_warp(o_done(w), (it - 1) & 1)) {
-          failed = true;
-          break;
-        }
-        tc::fence_after();
+        // this stream's previous PV is done (it was issued before this tile's S, which
+        // has completed): O may be rescaled
         if (any_need) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -388,11 +389,11 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
       tc::fence_before();
       tc::mbar_arrive(p_full(w));
     }
-    // this stream's last PV
+    // this stream's last PV (o_done is committed once per stream)
     const bool had = !failed && it > 0;
     bool have_o = false;
     if (had) {
-      if (wait_warp(o_done(w), (it - 1) & 1)) {
+      if (wait_warp(o_done(w), 0)) {
         tc::fence_after();
         have_o = true;
       } else {
