@@ -92,7 +92,10 @@ def test_full_size_forward_path(name):
     assert gm.sum(-1).min() >= 1
 
 
-def test_full_size_backward_wan14b():
+@pytest.mark.parametrize("pair", ["exact", "training"])
+def test_full_size_backward_wan14b(pair):
+    """The backward at the Wan-14B shape: the exact one (D pass) and the training pair
+    (the training forward's fp32 O gives D)."""
     wl = WORKLOADS["wan-14b-720p"]
     x = make_inputs(wl, with_dout=True)
     perm = oracle.gilbert_order(wl.T, wl.Hg, wl.W)
@@ -107,8 +110,12 @@ def test_full_size_backward_wan14b():
     full = mask_from_csr(bm_gpu)
     full[:, h] = mask_h[:, 0]
     bm = upload_mask(full, wl.N)
-    o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
-    dq, dk, dv = asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm)
+    if pair == "exact":
+        o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
+        dq, dk, dv = asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm)
+    else:
+        o, lse, o32 = asa.asa_sparse_attn_fwd_train(qp, kp, vp, bm)
+        dq, dk, dv = asa.asa_sparse_attn_bwd_train(qp, kp, vp, o32, dop, lse, bm)
     torch.cuda.synchronize()
     asa.asa_check_device_status()
     # invariants at full size, every head
@@ -129,10 +136,10 @@ def test_full_size_backward_wan14b():
                                           q_blocks=q_blocks, kv_blocks=[J])
     for I in q_blocks:
         rows = slice(128 * I, min(128 * I + 128, wl.N))
-        check_close(f64(dq[0, h, rows]), dq_ref[(0, 0, I)], what=f"dQ block {I}")
+        check_close(f64(dq[0, h, rows]), dq_ref[(0, 0, I)], what=f"{pair} dQ block {I}")
     rows = slice(128 * J, min(128 * J + 128, wl.N))
-    check_close(f64(dk[0, h, rows]), dkv_ref[(0, 0, J)][0], what=f"dK block {J}")
-    check_close(f64(dv[0, h, rows]), dkv_ref[(0, 0, J)][1], what=f"dV block {J}")
+    check_close(f64(dk[0, h, rows]), dkv_ref[(0, 0, J)][0], what=f"{pair} dK block {J}")
+    check_close(f64(dv[0, h, rows]), dkv_ref[(0, 0, J)][1], what=f"{pair} dV block {J}")
 
 
 def test_full_size_backward_asa_g_wan():

@@ -1,9 +1,10 @@
 """The largest call the library accepts: N = ASA_MAX_TOKENS = 262,144 tokens (grid
 4 x 256 x 256, 2,048 blocks), one head, d = 64, through permute -> estimate + mask ->
-forward -> backward.  Checked on outputs the oracle can compute one by one: sampled
-permuted rows, P_imp and mask rows of sampled query blocks (the oracle computes only
-those rows), forward rows of those blocks, dQ of sampled blocks, and the backward's
-invariants over the whole call."""
+forward -> backward, and through the training pair.  Checked on outputs the oracle can
+compute one by one: sampled permuted rows, P_imp and mask rows of sampled query blocks
+(the oracle computes only those rows; a row that differs must be marginal and a legal
+cut), forward rows of those blocks and their dQ under the library's rows, and the
+backward's invariants over the whole call."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,7 @@ import torch
 import oracle
 from inputs import WORKLOADS, make_inputs
 from video_dit_dynamic_gilbert_b200 import asa
-from gpu_util import check_close, f64, mask_from_csr
+from gpu_util import check_close, compare_masks, f64, mask_from_csr
 
 pytestmark = pytest.mark.gpu
 
@@ -29,6 +30,8 @@ def test_max_tokens_end_to_end():
     bm = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
     o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm)
     dq, dk, dv = asa.asa_sparse_attn_bwd(qp, kp, vp, o, dop, lse, bm)
+    o_t, lse_t, o32 = asa.asa_sparse_attn_fwd_train(qp, kp, vp, bm)
+    dq_t, dk_t, dv_t = asa.asa_sparse_attn_bwd_train(qp, kp, vp, o32, dop, lse_t, bm)
     torch.cuda.synchronize()
     asa.asa_check_device_status()
     assert torch.equal(asa.asa_unpermute(qp, wl.T, wl.Hg, wl.W), q)
@@ -46,23 +49,25 @@ def test_max_tokens_end_to_end():
     gm = mask_from_csr(bm)[:, :, blocks]
     mask_rows = oracle.build_mask(pimp_rows, wl.tau)
     marg = oracle.marginal_rows(pimp_rows, wl.tau)
-    differ = (gm != mask_rows).any(-1)
-    assert not (differ & ~marg).any()
-    agree = [I for I, dif in zip(blocks, differ[0, 0]) if not dif]
-    assert agree
+    compare_masks(gm, mask_rows, marg, pimp_rows, wl.tau, what="max size")
     full = np.zeros((1, 1, nb, nb), dtype=bool)
-    for I, row in zip(blocks, mask_rows[0, 0]):
+    for I, row in zip(blocks, gm[0, 0]):
         full[0, 0, I] = row
-    # forward rows and dQ of the agreeing blocks
+    # forward rows and dQ of the sampled blocks under the library's (legal) rows
     rows = np.concatenate([128 * I + g.choice(min(128, wl.N - 128 * I), 16, replace=False)
-                           for I in agree])
+                           for I in blocks])
     O_ref, L_ref = oracle.asa_forward(qh, kh, vh, full, q_index=rows)
     check_close(f64(o[0, 0, torch.from_numpy(rows)]), O_ref[0, 0], what="O at max size")
-    dq_ref, _ = oracle.asa_backward(qh, kh, vh, doh, full, heads=[(0, 0)], q_blocks=agree,
+    check_close(f64(o_t[0, 0, torch.from_numpy(rows)]), O_ref[0, 0],
+                what="O at max size (training forward)")
+    dq_ref, _ = oracle.asa_backward(qh, kh, vh, doh, full, heads=[(0, 0)], q_blocks=blocks,
                                     kv_blocks=[])
-    for I in agree:
+    for I in blocks:
         r = slice(128 * I, min(128 * I + 128, wl.N))
         check_close(f64(dq[0, 0, r]), dq_ref[(0, 0, I)], what=f"dQ block {I} at max size")
+        check_close(f64(dq_t[0, 0, r]), dq_ref[(0, 0, I)],
+                    what=f"dQ block {I} at max size (training pair)")
+    assert torch.equal(dv_t.view(torch.int16), dv.view(torch.int16))
     # invariants of the whole backward
     sum_dv, sum_do = dv.double().sum(dim=2), dop.double().sum(dim=2)
     scale = dop.double().abs().sum(dim=2).clamp_min(1.0)
