@@ -1,6 +1,7 @@
 """Seeded random small shapes through every step against the oracle: permutation
-(bit-exact), P_imp, mask rows (bit-exact unless marginal), forward and backward under
-the oracle's mask, for ASA and ASA_G.  Shapes cover single tokens, ragged last blocks,
+(bit-exact), P_imp, mask rows (bit-exact unless marginal, then a legal cut), forward
+and backward under the oracle's mask (the exact backward and the training pair), for
+ASA and ASA_G.  Shapes cover single tokens, ragged last blocks,
 blocks shorter than k = 16, batch 2, several heads, d = 64 and 128."""
 import math
 
@@ -11,7 +12,7 @@ import torch
 import oracle
 from inputs import WORKLOADS, make_inputs
 from video_dit_dynamic_gilbert_b200 import asa
-from gpu_util import check_close, f64, mask_from_csr, upload_mask
+from gpu_util import check_close, compare_masks, f64, mask_from_csr, upload_mask
 
 pytestmark = pytest.mark.gpu
 
@@ -45,7 +46,7 @@ def test_fuzz_whole_path(c):
     bm = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
     mask = oracle.build_mask(pimp, wl.tau)
     marg = oracle.marginal_rows(pimp, wl.tau)
-    assert not (((mask_from_csr(bm) != mask).any(-1)) & ~marg).any()
+    compare_masks(mask_from_csr(bm), mask, marg, pimp, wl.tau, what=f"fuzz seed {c['seed']}")
     # forward and backward under the oracle's mask
     bmo = upload_mask(mask, wl.N)
     o, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bmo, global_window=n)
@@ -69,6 +70,13 @@ def test_fuzz_whole_path(c):
     check_close(dq, rq, what="dQ")
     check_close(dk, rk, what="dK")
     check_close(dv, rv, what="dV")
+    # the training pair: D from the training forward's fp32 O
+    o_t, lse_t, o32 = asa.asa_sparse_attn_fwd_train(qp, kp, vp, bmo, global_window=n)
+    check_close(f64(o_t), O_ref, what="O (training forward)")
+    grads_t = asa.asa_sparse_attn_bwd_train(qp, kp, vp, o32, dop, lse_t, bmo, global_window=n)
+    asa.asa_check_device_status()
+    for g, r, nm in zip(grads_t, (rq, rk, rv), ("dQ", "dK", "dV")):
+        check_close(f64(g), r, what=f"{nm} (training pair)")
     # the raster output of the whole call
     out = asa.asa_unpermute(o, wl.T, wl.Hg, wl.W)
     check_close(f64(out)[:, perm].transpose(0, 2, 1, 3), O_ref, what="O raster")
