@@ -413,6 +413,20 @@ def _report_config(asa, torch, wl, timer, dev, peaks):
         tb = r["attn_bwd"]["median_ms"] * 1e-3
         r["attn_bwd"]["effective_TFLOP_s"] = 2.5 * flops / tb / 1e12
         r["attn_bwd"]["executed_TFLOP_s"] = 4.5 * flops / tb / 1e12
+        # the training pair: its forward (fp16 P V, fp32 O written) and its backward (D
+        # from that O, no D pass: 7 executed GEMM units per kept tile, i.e. 3.5 forwards)
+        tws = asa.fwd_train_workspace(B, H, N, d, gw, dev)
+        o_t, lse_t = torch.empty_like(qp), torch.empty_like(lse)
+        o32 = torch.empty(qp.shape, dtype=torch.float32, device=dev)
+        r["attn_fwd_train"] = timer(lambda: asa.asa_sparse_attn_fwd_train(
+            qp, kp, vp, mask, global_window=gw, workspace=tws, out=o_t, lse=lse_t, out32=o32))
+        r["attn_fwd_train"]["TFLOP_s"] = flops / (r["attn_fwd_train"]["median_ms"] * 1e-3) / 1e12
+        r["attn_bwd_train"] = timer(lambda: asa.asa_sparse_attn_bwd_train(
+            qp, kp, vp, o32, dop, lse_t, mask, global_window=gw, workspace=bws, outs=grads),
+            reps=8, warm=3)
+        tt = r["attn_bwd_train"]["median_ms"] * 1e-3
+        r["attn_bwd_train"]["effective_TFLOP_s"] = 2.5 * flops / tt / 1e12
+        r["attn_bwd_train"]["executed_TFLOP_s"] = 3.5 * flops / tt / 1e12
     # BSA query pruning with token filling on the same mask: r = 0.5, windows of 8
     pr = asa.asa_prune_queries(qp, 0.5, 8)
     pmws = asa._workspace(asa.lib().asa_prune_mask_workspace_size(B, H, N, pr.pack), dev)
@@ -558,6 +572,9 @@ def run_report(path):
         if "attn_bwd" in r:
             line += (f" bwd {r['attn_bwd']['median_ms']:.2f} ms "
                      f"{r['attn_bwd']['effective_TFLOP_s']:.0f} TF/s eff")
+        if "attn_bwd_train" in r:
+            line += (f" bwd_train {r['attn_bwd_train']['median_ms']:.2f} ms "
+                     f"{r['attn_bwd_train']['effective_TFLOP_s']:.0f} TF/s eff")
         qpr = r["query_prune"]
         line += (f" | pruned r=0.5: fwd {qpr['attn_fwd']['median_ms']:.3f} ms "
                  f"(x{qpr['fwd_speedup']:.2f})")

@@ -607,8 +607,9 @@ class ASAAttention(torch.autograd.Function):
     differentiated (the pages fix it for training as for inference); the backward runs
     under that mask, its gradients unpermuted to raster layout.  Without query pruning
     the forward is asa_sparse_attn_fwd_train and the backward asa_sparse_attn_bwd_train
-    (D from the fp32 O); d_from_o=True takes the inference forward and
-    asa_sparse_attn_bwd_d_from_o instead; with query_keep the pruned pair."""
+    (D from the fp32 O, which the op keeps between the two: 4 bytes per element of O);
+    d_from_o=True takes the inference forward and asa_sparse_attn_bwd_d_from_o instead;
+    with query_keep the pruned pair."""
 
     @staticmethod
     def forward(ctx, q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
