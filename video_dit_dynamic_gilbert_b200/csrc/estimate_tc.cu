@@ -9,13 +9,14 @@
 //   est_gather   compact Q_s, K_s [BH][Mp][d] (row 16 I + j = sample j of block I;
 //                rows past a short last block and past 16 nb are zero);
 //   est_tc       one CTA per (head, 128 sample rows, chunk of 128-column tiles):
-//                S = Q_s K_s^T tiles on tcgen05 into a double-buffered TMEM S, one
-//                softmax warpgroup (thread = sample row) writes each 16-column group's
-//                max logit G[bh, J, r] and keeps the row's online (max, sum) for its
-//                chunk;
-//   est_combine  lse2[bh, r] from the chunks' (max, sum);
+//                S = Q_s K_s^T tiles on tcgen05 into a double-buffered TMEM S; two
+//                softmax warpgroups split every tile's columns (warpgroup w takes
+//                [64 w, 64 w + 64); thread = sample row): each writes its 16-column
+//                groups' max logit G[bh, J, r] and keeps the row's online (max, sum)
+//                over its half of the chunk;
+//   est_combine  lse2[bh, r] from the (max, sum) of every chunk half;
 //   est_pool     P_imp[bh, I, J] = max_{r in I} exp2(G[bh, J, r] - lse2[bh, r]).
-// 6 warps and 256 TMEM columns per CTA, two CTAs per SM.
+// 10 warps and 256 TMEM columns per CTA, two CTAs per SM.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -29,7 +30,8 @@ bool make_map_rows(CUtensorMap* m, const void* ptr, int BH, int rows, int D);
 
 namespace {
 
-constexpr int kEstThreads = 192;      // producer, MMA, one softmax warpgroup
+constexpr int kEstThreads = 320;      // producer, MMA, two softmax warpgroups
+constexpr int kEstHalves = 2;         // softmax warpgroups, each a partial (max, sum) per row
 constexpr uint32_t kEstTmemCols = 256;  // two 128-column S buffers
 constexpr int kEstStages = 2;
 constexpr int kTilesPerChunk = 8;     // 128-column tiles per CTA
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kEstThreads, 2)
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full(b), 1);
-      tc::mbar_init(s_empty(b), 128);
+      tc::mbar_init(s_empty(b), 128 * kEstHalves);
     }
     tc::mbar_init(drain, 1);
     tc::fence_barrier_init();
@@ -185,11 +187,12 @@ __global__ void __launch_bounds__(kEstThreads, 2)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int quarter = warp & 3;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int w = (warp - 2) >> 2;  // warps 2-5: columns [0, 64); warps 6-9: [64, 128)
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const int r = 128 * mt + row;  // sample row of the head
-    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 64u * w;
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < ntile; ++j) {
       const int b = j & 1;
@@ -199,25 +202,25 @@ __global__ void __launch_bounds__(kEstThreads, 2)
         break;
       }
       tc::fence_after();
-      uint32_t s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32(trow + 128u * b + 32u * c, s + 32 * c);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_wait_ld_dep32(s + 32 * c);
-      // the buffer is free for the tile after next as soon as it is in registers
+      uint32_t s[64];
+      tc::tmem_ld32(trow + 128u * b, s);
+      tc::tmem_ld32(trow + 128u * b + 32u, s + 32);
+      tc::tmem_wait_ld_dep32(s);
+      tc::tmem_wait_ld_dep32(s + 32);
+      // the buffer is free for the tile after next as soon as both halves are in registers
       tc::fence_before();
       tc::mbar_arrive(s_empty(b));
-      const int nt = t0 + j;          // column tile
-      const int nvalid = M - 128 * nt;  // valid sample columns in this tile
-      if (nvalid < 128) {
+      const int nt = t0 + j;                   // column tile
+      const int nvalid = M - 128 * nt - 64 * w;  // valid sample columns in this half
+      if (nvalid < 64) {
 #pragma unroll
-        for (int k = 0; k < 128; ++k)
+        for (int k = 0; k < 64; ++k)
           if (k >= nvalid) s[k] = __float_as_uint(-INFINITY);
       }
       // block maxima (raw scores; c2 > 0 keeps the order) and the row max
-      float gm[8];
+      float gm[4];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 4; ++g) {
         float a = max3f(__uint_as_float(s[16 * g]), __uint_as_float(s[16 * g + 1]),
                         __uint_as_float(s[16 * g + 2]));
         float bq = max3f(__uint_as_float(s[16 * g + 3]), __uint_as_float(s[16 * g + 4]),
@@ -229,27 +232,28 @@ __global__ void __launch_bounds__(kEstThreads, 2)
         }
         gm[g] = max3f(a, bq, fmaxf(__uint_as_float(s[16 * g + 14]), __uint_as_float(s[16 * g + 15])));
       }
-      const float mraw = fmaxf(max3f(max3f(gm[0], gm[1], gm[2]), max3f(gm[3], gm[4], gm[5]), gm[6]), gm[7]);
+      const float mraw = fmaxf(max3f(gm[0], gm[1], gm[2]), gm[3]);
       if (r < M) {
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const int J = 8 * nt + g;
+        for (int g = 0; g < 4; ++g) {
+          const int J = 8 * nt + 4 * w + g;
           if (J < nb) G[(static_cast<int64_t>(bh) * nb + J) * (kSamples * nb) + r] = gm[g] * c2;
         }
       }
-      const float m_new = fmaxf(m, mraw * c2);  // finite: every tile has a valid column
-      const float mu = m_new;
-      const uint64_t c2x2 = f2_pack(c2, c2), offx2 = f2_pack(-mu, -mu);
+      // a half with no valid column (the last tile's) keeps its running (max, sum)
+      if (mraw == -INFINITY) continue;
+      const float m_new = fmaxf(m, mraw * c2);
+      const uint64_t c2x2 = f2_pack(c2, c2), offx2 = f2_pack(-m_new, -m_new);
       uint64_t rs = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
+      for (int k = 0; k < 32; ++k) {
         const uint64_t x2 =
             f2_fma(f2_pack(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2x2, offx2);
         float a, bq;
         if ((k & 3) == 0) {
           exp2_fma2(x2, a, bq);
           // exp2_fma clamps at -125: keep masked columns at zero
-          if (nvalid < 128) {
+          if (nvalid < 64) {
             a = 2 * k < nvalid ? a : 0.f;
             bq = 2 * k + 1 < nvalid ? bq : 0.f;
           }
@@ -266,7 +270,9 @@ __global__ void __launch_bounds__(kEstThreads, 2)
       l = l * fast_exp2(m - m_new) + (ra + rb);
       m = m_new;
     }
-    if (r < Mp) part[(static_cast<int64_t>(bh) * nchunk + chunk) * Mp + r] = make_float2(m, l);
+    if (r < Mp)
+      part[(static_cast<int64_t>(bh) * nchunk * kEstHalves + kEstHalves * chunk + w) * Mp + r] =
+          make_float2(m, l);
   }
 
   if (failed) atomicOr(err_word, 2u);
@@ -355,7 +361,7 @@ cudaError_t launch_est_tc(const void* qs, const void* ks, int BH, int N, int nb,
   if (e != cudaSuccess) return e;
   const int Mpad16 = kSamples * nb;
   est_combine_kernel<<<grid_cap(static_cast<int64_t>(BH) * Mpad16, 256, num_sms, 16), 256, 0,
-                       stream>>>(part, lse2, BH, Mp, Mpad16, nchunk);
+                       stream>>>(part, lse2, BH, Mp, Mpad16, nchunk * kEstHalves);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   est_pool_kernel<<<grid_cap(static_cast<int64_t>(BH) * nb * nb, 256, num_sms, 16), 256, 0,
@@ -371,7 +377,7 @@ size_t est_scratch_floats(int BH, int nb) {
   const size_t nchunk = (ntn + kTilesPerChunk - 1) / kTilesPerChunk;
   return static_cast<size_t>(BH) * nb * kSamples * nb   // G
          + static_cast<size_t>(BH) * kSamples * nb      // lse2
-         + static_cast<size_t>(BH) * nchunk * Mp * 2    // per-chunk (max, sum)
+         + static_cast<size_t>(BH) * nchunk * kEstHalves * Mp * 2  // per chunk half (max, sum)
          + 2 * static_cast<size_t>(BH) * Mp * 128 / 2   // Q_s, K_s (bf16, d <= 128)
          + 64;                                          // alignment of Q_s
 }
@@ -387,7 +393,8 @@ cudaError_t launch_estimate(const void* qp, const void* kp, int BH, int N, int d
   float* lse2 = G + static_cast<size_t>(BH) * nb * kSamples * nb;
   float2* part = reinterpret_cast<float2*>(lse2 + static_cast<size_t>(BH) * kSamples * nb);
   // Q_s, K_s at a 16-byte boundary after the partial sums
-  uintptr_t qa = reinterpret_cast<uintptr_t>(part + static_cast<size_t>(BH) * nchunk * Mp);
+  uintptr_t qa =
+      reinterpret_cast<uintptr_t>(part + static_cast<size_t>(BH) * nchunk * kEstHalves * Mp);
   qa = (qa + 255) & ~static_cast<uintptr_t>(255);
   uint4* qs = reinterpret_cast<uint4*>(qa);
   uint4* ks = qs + static_cast<size_t>(BH) * Mp * d / 8;
