@@ -44,6 +44,8 @@ def count_launches(torch, step):
             torch.cuda.synchronize()
         names = [e.name for e in prof.events()
                  if "asa::" in e.name and str(e.device_type).endswith("CUDA")]
+        if not names:  # a step always launches kernels: another profiler holds CUPTI
+            return None, "profiler saw no kernels (CUPTI held by another profiler)"
         return len(names), sorted(set(n.split("(")[0][-60:] for n in names))
     except Exception as exc:  # noqa: BLE001 - report, do not fail the bench
         return None, f"profiler unavailable: {type(exc).__name__}"
