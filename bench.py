@@ -3,7 +3,8 @@
 
 A step is the whole hot path of one training-free ASA self-attention call on
 resident inputs: Gilbert permute of Q, K, V -> sampled block-importance estimate ->
-tau-threshold mask (CSR) -> block-sparse attention forward -> unpermute of O.
+tau-threshold mask (CSR) -> block-sparse attention forward, which stores O straight
+back to raster order (the inverse permutation fused into its store).
 Prints ONE JSON line (rank 0).  Metric: effective TFLOP/s counting only kept tiles
 (4 d sum_kept L_I L_J per head), whole-job (all ranks) over the max-over-ranks time.
 
@@ -644,7 +645,6 @@ def main():
     B, N, H, d = q.shape
     T, Hg, W = wl.T, wl.Hg, wl.W
     qp, kp, vp = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
-    op = torch.empty_like(qp)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     out = torch.empty_like(q)
     ws = asa.estimate_mask_workspace(B, H, N, dev)
@@ -663,12 +663,10 @@ def main():
         asa.asa_estimate_mask(qp, kp, wl.tau, transposed=False, workspace=ws, mask=mask)
         if marks is not None:
             marks[2].record(stream)
-        asa.asa_sparse_attn_fwd(qp, kp, vp, mask, workspace=fws, out=op, lse=lse)
+        asa.asa_sparse_attn_fwd_raster(qp, kp, vp, mask, T, Hg, W, workspace=fws, out=out,
+                                       lse=lse)
         if marks is not None:
             marks[3].record(stream)
-        asa.asa_unpermute(op, T, Hg, W, out=out)
-        if marks is not None:
-            marks[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -678,7 +676,7 @@ def main():
 
     clocks = ClockSampler(local)
     time.sleep(0.3)
-    marks = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
     start, stop = ev(), ev()
     if world > 1:
         dist.barrier()
@@ -692,7 +690,7 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     elapsed_ms = start.elapsed_time(stop)
-    stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(4)] for m in marks])
+    stage = np.array([[m[j].elapsed_time(m[j + 1]) for j in range(3)] for m in marks])
     st_ms = stage.mean(axis=0)
     fwd_ms = float(st_ms[2])
 
@@ -704,7 +702,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": _config(wl),
         "stages_ms": {"permute_qkv": float(st_ms[0]), "estimate_mask": float(st_ms[1]),
-                      "attn_fwd": fwd_ms, "unpermute": float(st_ms[3])},
+                      "attn_fwd": fwd_ms},
         "kept_tiles": nnz, "tiles": tiles, "kept_fraction": nnz / tiles,
         "effective_flops_per_call": flops,
         "roofline": {"kernel": "asa sparse attention forward", "bound": "tensor",

@@ -204,6 +204,22 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
                         void* stream);
 
 /*
+ * asa_sparse_attn_fwd followed by the inverse Gilbert permutation (Preprocessing: the
+ * output returns to the original token order), fused: each output row is stored
+ * straight to its raster position, o[b, perm[i], h, :] = O[b, h, i, :], so no permuted
+ * O is written.  N = T*Hg*W; qp, kp, vp, the CSR, workspace (asa_fwd_workspace_size)
+ * and lse (device fp32 [B, H, N], Gilbert order) as in asa_sparse_attn_fwd;
+ * o: device bf16 [B, N, H, d] (raster layout, as asa_unpermute writes), not aliasing
+ * an input.  The result is bit-identical to asa_sparse_attn_fwd then asa_unpermute.
+ * Errors as asa_sparse_attn_fwd, plus ASA_ERR_INVALID_ARG for a bad grid.
+ */
+int asa_sparse_attn_fwd_raster(const void* qp, const void* kp, const void* vp,
+                               const int32_t* row_ptr, const int32_t* col_idx, int B, int T,
+                               int Hg, int W, int H, int d, int block, int global_window,
+                               void* workspace, size_t ws_bytes, void* o, float* lse,
+                               void* stream);
+
+/*
  * Workspace bytes of asa_sparse_attn_fwd_train (0 for invalid sizes): those of
  * asa_sparse_attn_fwd plus an fp16 copy of V (B*H*N*d * 2 bytes) and, with
  * global_window = n > 0, an fp16 copy of the G global V tokens (B*H*G*d * 2 bytes).

@@ -244,8 +244,9 @@ def test_host_call_rejects(L):
 
 
 def test_host_call_workspace_sizes(L):
-    # two slots of head_chunk heads: 8 raster/permuted tensors of B*hc*N*d bf16 each, plus
-    # the per-chunk estimator, mask and forward workspaces
+    # two slots of head_chunk heads: 7 raster/permuted tensors of B*hc*N*d bf16 each (Q, K,
+    # V in both orders and the raster O, which the forward stores directly), plus the
+    # per-chunk estimator, mask and forward workspaces
     B, T, Hg, W, H, d = 1, 21, 30, 52, 12, 128
     N = T * Hg * W
     one = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 1)
@@ -253,7 +254,8 @@ def test_host_call_workspace_sizes(L):
     assert one == L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0)     # ceil(12/12)
     assert L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 0) == \
         L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 4)               # ceil(48/12)
-    assert one >= 2 * 8 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
+    assert one >= 2 * 7 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
+    assert one < 2 * 8 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
     assert 2.5 * one < three < 3.5 * one
     assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 99) == \
         L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, H)
@@ -324,6 +326,20 @@ def test_training_pair_rejects(L):
     bargs[3] = MIS
     assert L.asa_sparse_attn_bwd_train(*bargs) == asa.ASA_ERR_INVALID_ARG
     assert b"o32" in L.asa_last_error_string()
+
+
+def test_fwd_raster_rejects(L):
+    # grid 4 x 16 x 16 = 1024 tokens, B=1, H=2
+    def call(T=4, d=64, o=FAKE, gw=0, ws=None, wsb=0, vp=FAKE):
+        return L.asa_sparse_attn_fwd_raster(FAKE, FAKE, vp, FAKE, FAKE, 1, T, 16, 16, 2, d, 128,
+                                            gw, ws, wsb, o, FAKE, None)
+    assert call(T=0) == asa.ASA_ERR_INVALID_ARG
+    assert call(d=96) == asa.ASA_ERR_UNSUPPORTED
+    assert call(o=FAKE) == asa.ASA_ERR_INVALID_ARG            # o aliases qp
+    other = ctypes.c_void_p(0x20000)
+    assert call(o=other, gw=-1) == asa.ASA_ERR_INVALID_ARG
+    assert call(o=other) == asa.ASA_ERR_WORKSPACE
+    assert call(o=other, vp=MIS) == asa.ASA_ERR_INVALID_ARG
 
 
 def test_global_pool_kv_rejects(L):

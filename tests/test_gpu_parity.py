@@ -160,6 +160,24 @@ def test_forward_with_oracle_mask(name):
     check_close(f64(lse), L_ref, max_abs=LSE_ABS, rel_l2=1e-4, what="LSE")
 
 
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("n", [0, 64])
+def test_forward_raster_is_forward_then_unpermute(name, n):
+    """The forward that stores O straight to raster order equals the forward followed by
+    the unpermute, bit for bit, and writes every element (the output starts as NaN)."""
+    wl, x, perm, ref, pimp, mask, marg, dev = setup_case(name)
+    qp, kp, vp = asa.asa_gilbert_permute3(dev["q"], dev["k"], dev["v"], wl.T, wl.Hg, wl.W)
+    bm = upload_mask(mask, wl.N)
+    op, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm, global_window=n)
+    want = asa.asa_unpermute(op, wl.T, wl.Hg, wl.W)
+    out = torch.full_like(dev["q"], float("nan"))
+    got, lse_r = asa.asa_sparse_attn_fwd_raster(qp, kp, vp, bm, wl.T, wl.Hg, wl.W,
+                                                global_window=n, out=out)
+    asa.asa_check_device_status()
+    assert torch.equal(got, want)
+    assert torch.equal(lse_r, lse)
+
+
 @pytest.mark.parametrize("name", ["tiny", "d128-ragged", "tail-lt-k"])
 def test_forward_dense_tau_one(name):
     wl, x, perm, ref, *_ = setup_case(name)

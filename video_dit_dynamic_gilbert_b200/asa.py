@@ -42,6 +42,7 @@ _SIGNATURES = {
     "asa_global_pool_kv": ([_vp] * 4 + [_c_int] * 5 + [_vp], _c_int),
     "asa_fwd_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_fwd": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
+    "asa_sparse_attn_fwd_raster": ([_vp] * 5 + [_c_int] * 8 + [_vp, _c_size, _vp, _vp, _vp], _c_int),
     "asa_fwd_train_workspace_size": ([_c_int] * 5, _c_size),
     "asa_sparse_attn_fwd_train": ([_vp] * 5 + [_c_int] * 6 + [_vp, _c_size, _vp, _vp, _vp, _vp],
                                   _c_int),
@@ -331,6 +332,28 @@ def asa_sparse_attn_fwd(qp, kp, vp, mask: BlockMask, global_window: int = 0, wor
     return out, lse
 
 
+def asa_sparse_attn_fwd_raster(qp, kp, vp, mask: BlockMask, T: int, Hg: int, W: int,
+                               global_window: int = 0, workspace=None, out=None, lse=None,
+                               stream=None):
+    """asa_sparse_attn_fwd with the inverse Gilbert permutation fused into its store:
+    O in raster layout [B, N, H, d] bf16 (as asa_unpermute returns it) and LSE
+    [B, H, N] fp32 in Gilbert order."""
+    for n_, t in (("qp", qp), ("kp", kp), ("vp", vp)):
+        _bf16_cuda(n_, t)
+    B, H, N, d = qp.shape
+    if workspace is None:
+        workspace = fwd_workspace(B, H, N, d, global_window, qp.device)
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=qp.dtype, device=qp.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=qp.device)
+    _check(lib().asa_sparse_attn_fwd_raster(_ptr(qp), _ptr(kp), _ptr(vp), _ptr(mask.row_ptr),
+                                            _ptr(mask.col_idx), B, T, Hg, W, H, d, BLOCK,
+                                            global_window, _ptr(workspace), _ws_bytes(workspace),
+                                            _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
 def fwd_train_workspace(B, H, N, d, global_window, device):
     return _workspace(lib().asa_fwd_train_workspace_size(B, H, N, d, global_window), device)
 
@@ -559,13 +582,15 @@ def asa_shutdown() -> None:
 def asa_attention(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
                   query_keep: float | None = None, query_window: int = 8, stream=None):
     """One ASA self-attention call on raster-layout q, k, v [B, N, H, d]: Gilbert permute,
-    estimate + mask, block-sparse forward, unpermute.  Returns (O raster, LSE, mask).
-    query_keep = r adds BSA's query pruning with token filling (windows of
-    query_window permuted tokens)."""
+    estimate + mask, block-sparse forward storing O straight back to raster order.
+    Returns (O raster, LSE in Gilbert order, mask).  query_keep = r adds BSA's query
+    pruning with token filling (windows of query_window permuted tokens)."""
     qp, kp, vp = asa_gilbert_permute3(q, k, v, T, Hg, W, stream=stream)
     mask = asa_estimate_mask(qp, kp, tau, transposed=False, stream=stream)
     if query_keep is None:
-        op, lse = asa_sparse_attn_fwd(qp, kp, vp, mask, global_window=global_window, stream=stream)
+        out, lse = asa_sparse_attn_fwd_raster(qp, kp, vp, mask, T, Hg, W,
+                                              global_window=global_window, stream=stream)
+        return out, lse, mask
     else:
         prune = asa_prune_queries(qp, query_keep, query_window, stream=stream)
         tmask = asa_prune_mask(mask, prune.pack, stream=stream)

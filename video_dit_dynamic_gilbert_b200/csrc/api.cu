@@ -403,10 +403,11 @@ size_t asa_fwd_workspace_size(int B, int H, int N, int d, int global_window) {
   return bytes;
 }
 
-int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
-                        const int32_t* col_idx, int B, int H, int N, int d, int block,
-                        int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
-                        void* stream) {
+// perm_out != nullptr: O in raster layout [B, N, H, d] (token perm_out[i] for row i)
+static int fwd_impl(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                    const int32_t* col_idx, int B, int H, int N, int d, int block,
+                    int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
+                    const int32_t* perm_out, void* stream) {
   ASA_TRY(check_common(B, H, N, d));
   ASA_TRY(check_block(block, ASA_SAMPLES));
   ASA_TRY(check_ptr(qp, "qp"));
@@ -439,9 +440,44 @@ int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const in
   cudaError_t e = device_error_word(&err_word);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
   e = asa::launch_fwd_tc(qp, kp, vp, row_ptr, col_idx, kg, vg, order, B * H, N, d, global_window, o,
-                         lse, err_word, s);
+                         lse, err_word, s, perm_out, H);
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
   return ASA_OK;
+}
+
+int asa_sparse_attn_fwd(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
+                        const int32_t* col_idx, int B, int H, int N, int d, int block,
+                        int global_window, void* workspace, size_t ws_bytes, void* o, float* lse,
+                        void* stream) {
+  return fwd_impl(qp, kp, vp, row_ptr, col_idx, B, H, N, d, block, global_window, workspace,
+                  ws_bytes, o, lse, nullptr, stream);
+}
+
+int asa_sparse_attn_fwd_raster(const void* qp, const void* kp, const void* vp,
+                               const int32_t* row_ptr, const int32_t* col_idx, int B, int T,
+                               int Hg, int W, int H, int d, int block, int global_window,
+                               void* workspace, size_t ws_bytes, void* o, float* lse,
+                               void* stream) {
+  int64_t N = 0;
+  ASA_TRY(check_grid(T, Hg, W, &N));
+  ASA_TRY(check_common(B, H, static_cast<int>(N), d));
+  ASA_TRY(check_block(block, ASA_SAMPLES));
+  ASA_TRY(check_ptr(qp, "qp"));
+  ASA_TRY(check_ptr(kp, "kp"));
+  ASA_TRY(check_ptr(vp, "vp"));
+  ASA_TRY(check_ptr(row_ptr, "row_ptr", false));
+  ASA_TRY(check_ptr(col_idx, "col_idx", false));
+  ASA_TRY(check_ptr(o, "o"));
+  ASA_TRY(check_ptr(lse, "lse", false));
+  if (o == qp || o == kp || o == vp) return fail(ASA_ERR_INVALID_ARG, "o aliases an input");
+  if (global_window < 0) return fail(ASA_ERR_INVALID_ARG, "global_window=%d < 0", global_window);
+  // every host-side check before the permutation table is looked up on the device
+  ASA_TRY(check_ws(workspace, ws_bytes,
+                   asa_fwd_workspace_size(B, H, static_cast<int>(N), d, global_window)));
+  const int32_t* perm = nullptr;
+  ASA_TRY(get_perm(T, Hg, W, &perm));
+  return fwd_impl(qp, kp, vp, row_ptr, col_idx, B, H, static_cast<int>(N), d, block,
+                  global_window, workspace, ws_bytes, o, lse, perm, stream);
 }
 
 size_t asa_fwd_train_workspace_size(int B, int H, int N, int d, int global_window) {
@@ -796,7 +832,6 @@ int host_chunk(int H, int head_chunk) {
 struct HostSlot {
   char* x[3];
   char* xp[3];
-  char* op;
   char* out;
   char* est_ws;
   size_t est_bytes;
@@ -820,7 +855,6 @@ HostSlot carve_host_slot(char* base, int B, int hc, int N, int d, int global_win
   const size_t rows = static_cast<size_t>(B) * hc * nb;
   for (int i = 0; i < 3; ++i) r.x[i] = take(t);
   for (int i = 0; i < 3; ++i) r.xp[i] = take(t);
-  r.op = take(t);
   r.out = take(t);
   r.est_bytes = asa_estimate_mask_workspace_size(B, hc, N);
   r.est_ws = take(r.est_bytes);
@@ -921,9 +955,9 @@ int asa_attention_host(const void* q, const void* k, const void* v, int B, int T
       rc = asa_estimate_mask(S.xp[0], S.xp[1], B, hcur, N, d, ASA_BLOCK, ASA_SAMPLES, tau, S.est_ws,
                              S.est_bytes, S.row_ptr, S.col_idx, S.nnz, nullptr, nullptr, P.cmp);
     if (rc == ASA_OK)
-      rc = asa_sparse_attn_fwd(S.xp[0], S.xp[1], S.xp[2], S.row_ptr, S.col_idx, B, hcur, N, d,
-                               ASA_BLOCK, global_window, S.fwd_ws, S.fwd_bytes, S.op, S.lse, P.cmp);
-    if (rc == ASA_OK) rc = asa_unpermute(S.op, S.out, B, T, Hg, W, hcur, d, P.cmp);
+      rc = asa_sparse_attn_fwd_raster(S.xp[0], S.xp[1], S.xp[2], S.row_ptr, S.col_idx, B, T, Hg,
+                                      W, hcur, d, ASA_BLOCK, global_window, S.fwd_ws, S.fwd_bytes,
+                                      S.out, S.lse, P.cmp);
     if (rc != ASA_OK) return finish(rc);
     cudaEventRecord(cmp_done(c), P.cmp);
     // copy out

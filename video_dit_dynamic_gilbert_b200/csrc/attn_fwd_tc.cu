@@ -102,8 +102,8 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
                   const int32_t* __restrict__ col_idx, const uint8_t* __restrict__ quarters,
                   const int32_t* __restrict__ order, int N, int Nq, int nb, int G, float gbias2,
                   float c2, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                  float* __restrict__ o32, unsigned int* __restrict__ err_word,
-                  long long wait_limit) {
+                  float* __restrict__ o32, const int32_t* __restrict__ perm_out, int H,
+                  unsigned int* __restrict__ err_word, long long wait_limit) {
   using L = FwdTcLayout<D, NST>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -420,7 +420,16 @@ __global__ void __launch_bounds__(kFwdTcThreads, 1)
     const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
     // warpgroup w writes columns [D/2 w, D/2 w + D/2) of its rows
     const int q = q0 + row;
-    const int64_t orow_off = (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
+    int64_t orow_off;
+    if (perm_out != nullptr) {
+      // O straight into raster layout [B, N, H, D] (the inverse Gilbert permutation
+      // fused into the store): permuted row q is token perm_out[q] of head h
+      const int b = bh / H, h = bh - b * H;
+      const int tok = q < Nq ? __ldg(perm_out + q) : 0;
+      orow_off = ((static_cast<int64_t>(b) * Nq + tok) * H + h) * D + (D / 2) * w;
+    } else {
+      orow_off = (static_cast<int64_t>(bh) * Nq + (q < Nq ? q : 0)) * D + (D / 2) * w;
+    }
     __nv_bfloat16* orow = o + orow_off;
     const bool h0 = __all_sync(0xffffffffu, has_0) != 0 || __any_sync(0xffffffffu, has_0) != 0;
     const bool h1 = __any_sync(0xffffffffu, has_1) != 0;
@@ -578,8 +587,8 @@ namespace {
 template <int D, int NST, bool kPruned, bool kTrain>
 cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int32_t* col_idx,
                       const uint8_t* quarters, int32_t* order, int BH, int N, int Nq, int G,
-                      float gbias2, void* o, float* lse, float* o32, unsigned int* err_word,
-                      cudaStream_t stream) {
+                      float gbias2, void* o, float* lse, float* o32, const int32_t* perm_out,
+                      int H, unsigned int* err_word, cudaStream_t stream) {
   using L = FwdTcLayout<D, NST>;
   const int nb = (Nq + kBlock - 1) / kBlock;
   const float c2 = kLog2e / sqrtf(static_cast<float>(D));
@@ -602,7 +611,7 @@ cudaError_t launch_tc(const CUtensorMap* maps, const int32_t* row_ptr, const int
   if (e != cudaSuccess) return e;
   fwd_tc_kernel<D, NST, kPruned, kTrain><<<rows, kFwdTcThreads, L::kSmem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], row_ptr, col_idx, quarters, order, N, Nq, nb,
-      G, gbias2, c2, static_cast<__nv_bfloat16*>(o), lse, o32, err_word, limit);
+      G, gbias2, c2, static_cast<__nv_bfloat16*>(o), lse, o32, perm_out, H, err_word, limit);
   return cudaGetLastError();
 }
 
@@ -612,7 +621,8 @@ cudaError_t launch_fwd_any(const void* qp, const void* kp, const void* vp, const
                            const int32_t* col_idx, const uint8_t* quarters, const void* kg,
                            const void* vg, int32_t* order, int BH, int N, int Nq, int d,
                            int global_window, void* o, float* lse, float* o32,
-                           unsigned int* err_word, cudaStream_t stream) {
+                           unsigned int* err_word, cudaStream_t stream,
+                           const int32_t* perm_out = nullptr, int H = 1) {
   const int G = global_window > 0 ? (N + global_window - 1) / global_window : 0;
   const float gbias2 = global_window > 0 ? log2f(static_cast<float>(global_window)) : 0.f;
   const CUtensorMapDataType vtype =
@@ -630,9 +640,10 @@ cudaError_t launch_fwd_any(const void* qp, const void* kp, const void* vp, const
   }
   if (d == 128)
     return launch_tc<128, 3, kPruned, kTrain>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq,
-                                              G, gbias2, o, lse, o32, err_word, stream);
+                                              G, gbias2, o, lse, o32, perm_out, H, err_word,
+                                              stream);
   return launch_tc<64, 6, kPruned, kTrain>(maps, row_ptr, col_idx, quarters, order, BH, N, Nq, G,
-                                           gbias2, o, lse, o32, err_word, stream);
+                                           gbias2, o, lse, o32, perm_out, H, err_word, stream);
 }
 
 }  // namespace
@@ -640,9 +651,10 @@ cudaError_t launch_fwd_any(const void* qp, const void* kp, const void* vp, const
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
                           const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
                           int BH, int N, int d, int global_window, void* o, float* lse,
-                          unsigned int* err_word, cudaStream_t stream) {
+                          unsigned int* err_word, cudaStream_t stream, const int32_t* perm_out,
+                          int H) {
   return launch_fwd_any<false>(qp, kp, vp, row_ptr, col_idx, nullptr, kg, vg, order, BH, N, N, d,
-                               global_window, o, lse, nullptr, err_word, stream);
+                               global_window, o, lse, nullptr, err_word, stream, perm_out, H);
 }
 
 cudaError_t launch_fwd_tc_train(const void* qp, const void* kp, const void* vp16,

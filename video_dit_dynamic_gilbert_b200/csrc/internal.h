@@ -57,10 +57,13 @@ cudaError_t launch_global_pool(const void* xp, void* xg, int BH, int N, int d, i
                                cudaStream_t stream, const void* xp2 = nullptr,
                                void* xg2 = nullptr);
 
+// perm_out != nullptr: O goes straight to raster layout [B, N, H, d], permuted row i of
+// head h to token perm_out[i] (BH = B * H); otherwise O is [BH][N][d] in Gilbert order
 cudaError_t launch_fwd_tc(const void* qp, const void* kp, const void* vp, const int32_t* row_ptr,
                           const int32_t* col_idx, const void* kg, const void* vg, int32_t* order,
                           int BH, int N, int d, int global_window, void* o, float* lse,
-                          unsigned int* err_word, cudaStream_t stream);
+                          unsigned int* err_word, cudaStream_t stream,
+                          const int32_t* perm_out = nullptr, int H = 1);
 
 // Training forward: PV with fp16 P and the fp16 copies vp16, vg16 of V and of the
 // global V tokens; writes O (bf16), LSE and the fp32 O.
