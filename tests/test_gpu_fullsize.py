@@ -30,15 +30,21 @@ FULL = ["wan2.1-1.3b", "cogvideox-5b", "wan2.1-1.3b-asag", "wan-14b-720p"]
 
 
 def _run(wl, x):
-    """The bench's call: permute Q,K,V -> estimate+mask -> forward -> unpermute."""
+    """The call: permute Q,K,V -> estimate+mask -> forward -> unpermute, and the bench's
+    forward that stores O straight to raster order (which must equal it bit for bit)."""
     q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
     qp, kp, vp = asa.asa_gilbert_permute3(q, k, v, wl.T, wl.Hg, wl.W)
     p_imp = asa.asa_estimate(qp, kp)
     bm = asa.asa_estimate_mask(qp, kp, wl.tau, transposed=True)
     op, lse = asa.asa_sparse_attn_fwd(qp, kp, vp, bm, global_window=wl.global_window)
     out = asa.asa_unpermute(op, wl.T, wl.Hg, wl.W)
+    out_r, lse_r = asa.asa_sparse_attn_fwd_raster(qp, kp, vp, bm, wl.T, wl.Hg, wl.W,
+                                                  global_window=wl.global_window)
     torch.cuda.synchronize()
     asa.asa_check_device_status()
+    assert torch.equal(out_r, out)
+    assert torch.equal(lse_r, lse)
+    del out_r, lse_r
     return dict(q=q, k=k, v=v, qp=qp, kp=kp, vp=vp, p_imp=p_imp, bm=bm, op=op, lse=lse, out=out)
 
 

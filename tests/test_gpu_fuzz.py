@@ -1,7 +1,7 @@
 """Seeded random small shapes through every step against the oracle: permutation
 (bit-exact), P_imp, mask rows (bit-exact unless marginal, then a legal cut), forward
-and backward under the oracle's mask (the exact backward and the training pair), for
-ASA and ASA_G.  Shapes cover single tokens, ragged last blocks,
+and backward under the oracle's mask (the exact backward and the training pair), the
+forward storing O straight to raster order, for ASA and ASA_G.  Shapes cover single tokens, ragged last blocks,
 blocks shorter than k = 16, batch 2, several heads, d = 64 and 128."""
 import math
 
@@ -77,6 +77,9 @@ def test_fuzz_whole_path(c):
     asa.asa_check_device_status()
     for g, r, nm in zip(grads_t, (rq, rk, rv), ("dQ", "dK", "dV")):
         check_close(f64(g), r, what=f"{nm} (training pair)")
-    # the raster output of the whole call
+    # the raster output of the whole call, and the forward that stores it directly
     out = asa.asa_unpermute(o, wl.T, wl.Hg, wl.W)
     check_close(f64(out)[:, perm].transpose(0, 2, 1, 3), O_ref, what="O raster")
+    out_r, lse_r = asa.asa_sparse_attn_fwd_raster(qp, kp, vp, bmo, wl.T, wl.Hg, wl.W,
+                                                  global_window=n)
+    assert torch.equal(out_r, out) and torch.equal(lse_r, lse)
