@@ -422,15 +422,16 @@ int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, 
  * ---------------------------------------------------------------------------- */
 
 /* Workspace bytes of asa_attention_host: two pipeline slots, each holding the device
- * copies of head_chunk heads (raster and permuted Q, K, V; permuted and raster O), the
+ * copies of head_chunk heads (raster and permuted Q, K, V; raster O), the
  * estimator and mask workspace and CSR, the forward workspace and the LSE of those
  * heads.  head_chunk = 0 takes ceil(H / 12).  0 for invalid sizes. */
 size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int d,
                                          int global_window, int head_chunk);
 
 /*
- * The whole call of asa_gilbert_permute3 -> asa_estimate_mask -> asa_sparse_attn_fwd
- * -> asa_unpermute (Preprocessing, Steps 1, 2.1, 2.2) for host buffers q, k, v, o
+ * The whole call of asa_gilbert_permute3 -> asa_estimate_mask ->
+ * asa_sparse_attn_fwd_raster (Preprocessing, Steps 1, 2.1, 2.2; the forward stores O
+ * straight to raster order) for host buffers q, k, v, o
  * (bf16 [B, T*Hg*W, H, d], raster order), in chunks of head_chunk heads (0: ceil(H/12),
  * one head per chunk up to 12 heads).
  * Chunk c's strided host-to-device copies, chunk c-1's kernels and chunk c-2's
