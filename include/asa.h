@@ -424,7 +424,7 @@ int asa_sparse_attn_bwd_pruned(const void* q_s, const void* kp, const void* vp, 
 /* Workspace bytes of asa_attention_host: two pipeline slots, each holding the device
  * copies of head_chunk heads (raster and permuted Q, K, V; raster O), the
  * estimator and mask workspace and CSR, the forward workspace and the LSE of those
- * heads.  head_chunk = 0 takes ceil(H / 12).  0 for invalid sizes. */
+ * heads.  head_chunk = 0 takes the default below.  0 for invalid sizes. */
 size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int d,
                                          int global_window, int head_chunk);
 
@@ -432,8 +432,9 @@ size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int
  * The whole call of asa_gilbert_permute3 -> asa_estimate_mask ->
  * asa_sparse_attn_fwd_raster (Preprocessing, Steps 1, 2.1, 2.2; the forward stores O
  * straight to raster order) for host buffers q, k, v, o
- * (bf16 [B, T*Hg*W, H, d], raster order), in chunks of head_chunk heads (0: ceil(H/12),
- * one head per chunk up to 12 heads).
+ * (bf16 [B, T*Hg*W, H, d], raster order), in chunks of head_chunk heads (0: the default,
+ * max(ceil(256/d), ceil(H/24)) heads, capped at H: host rows of at least 512 bytes in
+ * the strided copies, which narrower rows slow down, and at most 24 chunks).
  * Chunk c's strided host-to-device copies, chunk c-1's kernels and chunk c-2's
  * device-to-host copy run at once on three streams the library owns (one set per
  * device, released by asa_shutdown); two workspace slots alternate.  The call is

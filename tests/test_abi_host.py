@@ -251,9 +251,15 @@ def test_host_call_workspace_sizes(L):
     N = T * Hg * W
     one = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 1)
     three = L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 3)
-    assert one == L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0)     # ceil(12/12)
-    assert L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 0) == \
-        L.asa_attention_host_workspace_size(B, T, Hg, W, 48, d, 0, 4)               # ceil(48/12)
+    # default: max(ceil(256/d), ceil(H/24)) heads, capped at H
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 0) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, H, d, 0, 2)                # d=128, H=12
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, 48, 64, 0, 0) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, 48, 64, 0, 4)              # d=64
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, 96, d, 0, 0) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, 96, d, 0, 4)               # 24 chunks
+    assert L.asa_attention_host_workspace_size(B, T, Hg, W, 1, 64, 0, 0) == \
+        L.asa_attention_host_workspace_size(B, T, Hg, W, 1, 64, 0, 1)               # capped at H
     assert one >= 2 * 7 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
     assert one < 2 * 8 * N * d * 2 + 2 * L.asa_estimate_mask_workspace_size(B, 1, N)
     assert 2.5 * one < three < 3.5 * one

@@ -607,7 +607,8 @@ def host_workspace(B, T, Hg, W, H, d, global_window=0, head_chunk=0, device="cud
 def asa_attention_host(q, k, v, T: int, Hg: int, W: int, tau: float, global_window: int = 0,
                        head_chunk: int = 0, out=None, workspace=None, stream=None):
     """asa_attention on host (CPU) tensors q, k, v [B, N, H, d] bf16: the library copies
-    chunks of heads in (head_chunk = 0: ceil(H / 12) heads per chunk), computes and
+    chunks of heads in (head_chunk = 0: max(ceil(256 / d), ceil(H / 24)) heads per chunk,
+    capped at H), computes and
     copies O out, pipelined on its own streams; pin the
     tensors (tensor.pin_memory()) for the copies to overlap.  Returns O [B, N, H, d] on
     the host; synchronise the stream (torch.cuda.current_stream by default) before

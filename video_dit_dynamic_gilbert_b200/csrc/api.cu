@@ -823,8 +823,12 @@ struct HostPipe {
 std::mutex g_pipe_mu;
 std::map<int, HostPipe> g_pipes;
 
-int host_chunk(int H, int head_chunk) {
-  return head_chunk > 0 ? std::min(head_chunk, H) : std::max(1, (H + 11) / 12);
+// Default heads per chunk: at least 512 contiguous bytes per host row of a chunk's
+// strided copies (narrower rows copy markedly slower over PCIe), and at most 24
+// chunks (each chunk's copy and compute ends add fill and drain to the pipeline).
+int host_chunk(int H, int d, int head_chunk) {
+  if (head_chunk > 0) return std::min(head_chunk, H);
+  return std::min(H, std::max((256 + d - 1) / d, (H + 23) / 24));
 }
 
 // One slot of the pipeline: raster inputs, permuted inputs, permuted and raster
@@ -876,7 +880,7 @@ size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int
   if (B < 1 || H < 1 || T < 1 || Hg < 1 || W < 1 || N > ASA_MAX_TOKENS || (d != 64 && d != 128) ||
       global_window < 0 || head_chunk < 0)
     return 0;
-  const int hc = host_chunk(H, head_chunk);
+  const int hc = host_chunk(H, d, head_chunk);
   return 2 * carve_host_slot(nullptr, B, hc, static_cast<int>(N), d, global_window).bytes;
 }
 
@@ -894,7 +898,7 @@ int asa_attention_host(const void* q, const void* k, const void* v, int B, int T
   if (!(tau > 0.f)) return fail(ASA_ERR_INVALID_ARG, "tau=%g must be > 0", tau);
   ASA_TRY(check_ws(workspace, ws_bytes,
                    asa_attention_host_workspace_size(B, T, Hg, W, H, d, global_window, head_chunk)));
-  const int hc = host_chunk(H, head_chunk);
+  const int hc = host_chunk(H, d, head_chunk);
   const int nch = (H + hc - 1) / hc;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
