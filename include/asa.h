@@ -434,7 +434,8 @@ size_t asa_attention_host_workspace_size(int B, int T, int Hg, int W, int H, int
  * straight to raster order) for host buffers q, k, v, o
  * (bf16 [B, T*Hg*W, H, d], raster order), in chunks of head_chunk heads (0: the default,
  * max(ceil(256/d), ceil(H/24)) heads, capped at H: host rows of at least 512 bytes in
- * the strided copies, which narrower rows slow down, and at most 24 chunks).
+ * the strided copies, which narrower rows slow down, and at most 24 chunks; the last
+ * of two or more default chunks is split in two, shortening the pipeline's tail).
  * Chunk c's strided host-to-device copies, chunk c-1's kernels and chunk c-2's
  * device-to-host copy run at once on three streams the library owns (one set per
  * device, released by asa_shutdown); two workspace slots alternate.  The call is

@@ -899,7 +899,17 @@ int asa_attention_host(const void* q, const void* k, const void* v, int B, int T
   ASA_TRY(check_ws(workspace, ws_bytes,
                    asa_attention_host_workspace_size(B, T, Hg, W, H, d, global_window, head_chunk)));
   const int hc = host_chunk(H, d, head_chunk);
-  const int nch = (H + hc - 1) / hc;
+  // chunk c covers heads [ch0[c], ch0[c + 1]); with the default chunk size the last
+  // chunk is split in two, which halves the compute and copy-out that remain after
+  // the last copy-in
+  std::vector<int> ch0;
+  for (int h = 0; h < H; h += hc) ch0.push_back(h);
+  ch0.push_back(H);
+  if (head_chunk == 0 && ch0.size() > 2) {
+    const int a = ch0[ch0.size() - 2], last = H - a;
+    if (last >= 2) ch0.insert(ch0.end() - 1, a + (last + 1) / 2);
+  }
+  const int nch = static_cast<int>(ch0.size()) - 1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -940,7 +950,7 @@ int asa_attention_host(const void* q, const void* k, const void* v, int B, int T
   for (int c = 0; c < nch; ++c) {
     const HostSlot S = carve_host_slot(static_cast<char*>(workspace) + (c & 1) * slot_bytes, B, hc,
                                        N, d, global_window);
-    const int h0 = c * hc, hcur = std::min(hc, H - h0);
+    const int h0 = ch0[c], hcur = ch0[c + 1] - ch0[c];
     const size_t width = static_cast<size_t>(hcur) * d * 2;
     // copy in: the slot's inputs are free once chunk c - 2 has been computed
     if (c >= 2) cudaStreamWaitEvent(P.h2d, cmp_done(c - 2), 0);
